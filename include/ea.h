@@ -1,0 +1,187 @@
+/*
+ * ea.h — C ABI of the Elastic Attention prefill path for NVIDIA B200 (sm_100a).
+ *
+ * The method: "Elastic Attention: Test-time Adaptive Sparsity Ratios for
+ * Efficient Transformers" (arXiv 2601.17367; paperlayer.ai summary).  An
+ * Attention Router reads a layer's hidden states and gives every GQA key-value
+ * head a hard full / sparse decision (section 3 "Attention Router"); one
+ * hybrid-head attention launch then computes full causal heads and sparse
+ * heads (streaming sink + local window, or block-sparse) together and writes
+ * every head's output side by side (section 2 "Hybrid Head Mechanism";
+ * section 3 "Efficient Deployment"; appendix D.1 "Sparse Inference").
+ *
+ * Conventions for every call:
+ *  - Device pointers are CUDA device addresses on the current device; host
+ *    pointers are ordinary CPU memory.  The caller owns every buffer.  The
+ *    library never allocates device memory: scratch space is the caller's
+ *    `workspace`, sized by the matching *_workspace_size call, 256-byte
+ *    aligned, and zero-filled once before its first use (it keeps a sticky
+ *    device status word between calls).
+ *  - Layouts are row-major: q, o [B, S, H_q, d]; k, v [B, S, H_kv, d];
+ *    hidden [B, S, D].  Query head h_q reads KV head h_q / (H_q / H_kv).
+ *    q, k, v, o and hidden must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls enqueue work on it and return without waiting, except
+ *    ea_effective_sparsity and ea_workspace_status, which synchronise it.
+ *  - Errors: argument checks run on the host before any launch and return
+ *    EA_ERR_INVALID_ARG or EA_ERR_UNSUPPORTED with nothing enqueued.  A
+ *    failed launch returns EA_ERR_CUDA.  Problems only the device can see (a
+ *    malformed block layout or head_mode value, a pipeline wait that ran past
+ *    its time limit) set bits in the workspace status word; they surface on
+ *    the next ea_workspace_status / ea_effective_sparsity call on that
+ *    workspace as EA_ERR_BAD_LAYOUT or EA_ERR_TIMEOUT.
+ *  - Thread safety: calls that share a workspace must be ordered on one
+ *    stream.
+ */
+#ifndef EA_H_
+#define EA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define EA_API __attribute__((visibility("default")))
+#else
+#define EA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  EA_OK = 0,
+  EA_ERR_INVALID_ARG = 1,  /* a pointer, size or parameter is out of contract */
+  EA_ERR_UNSUPPORTED = 2,  /* valid, but not built (e.g. bf16 with d != 128)   */
+  EA_ERR_CUDA = 3,         /* a CUDA runtime or driver call failed             */
+  EA_ERR_TIMEOUT = 4,      /* a device pipeline wait ran out (status word)     */
+  EA_ERR_BAD_LAYOUT = 5    /* device-side check of head_mode / CSR failed      */
+} ea_status;
+
+typedef enum { EA_DT_F32 = 0, EA_DT_BF16 = 1 } ea_dtype;
+
+/* Head kinds (attention patterns).  FULL: keys 0..i.  STREAMING: keys j <= i
+ * with j < n_sink or i - j < window (sinks and the local window, united).
+ * BLOCK_SPARSE: keys j <= i whose block floor(j/block) is listed for the
+ * query block floor(i/block). */
+typedef enum { EA_FULL = 0, EA_STREAMING = 1, EA_BLOCK_SPARSE = 2 } ea_kind;
+
+/* Largest H_kv the calls accept (the per-head kind tables travel by value). */
+#define EA_MAX_KV_HEADS 64
+
+/* ------------------------------------------------------------------------
+ * Attention Router (section 3 "Attention Router"; appendix H.4 "Router
+ * Input Length"; section 5 "Attention Router" for the x4 MLP width).
+ *   hbar    = mean of hidden[b, t, :] over the pooled tokens: the first and
+ *             the last n_boundary tokens (every token once when
+ *             S <= 2 * n_boundary; the whole sequence when n_boundary <= 0)
+ *   p_h     = W_k[:, h*d:(h+1)*d]^T hbar                 (pooled key state)
+ *   tau_h   = W_t2 relu(W_t1 p_h + b_t1) + b_t2          (task MLP d->4d->d)
+ *   u_h     = relu(W_r1 [p_h; tau_h] + b_r1)              (router MLP 2d->4d)
+ *   z_h     = w_o[h] . u_h + b_o[h];  head_mode = (z_h > 0) (1 = sparse)
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int n_boundary; /* tokens pooled at each end; 100 by the pages; <= 0: all */
+} ea_router_params;
+
+typedef struct {          /* all device pointers, row-major                   */
+  const void* w_k;        /* [D, H_kv*d] key projection, in the hidden dtype  */
+  const float* w_t1;      /* [4d, d]   */
+  const float* b_t1;      /* [4d]      */
+  const float* w_t2;      /* [d, 4d]   */
+  const float* b_t2;      /* [d]       */
+  const float* w_r1;      /* [4d, 2d]  (input is [p; tau]) */
+  const float* b_r1;      /* [4d]      */
+  const float* w_o;       /* [H_kv, 4d] per-head output rows */
+  const float* b_o;       /* [H_kv]    */
+} ea_router_weights;
+
+/* Bytes of workspace ea_router needs (pooling partial sums and hbar). */
+EA_API size_t ea_router_workspace_size(int B, int S, int D, int n_boundary);
+
+/* Router for one layer.  hidden: device [B, S, D] in `dtype`
+ * (D % 8 == 0 for bf16, D % 4 == 0 for f32); d in {64, 128};
+ * 1 <= H_kv <= EA_MAX_KV_HEADS.  Writes head_mode [B, H_kv] (device int32,
+ * 0 dense / 1 sparse) and, when `logits` is not NULL, z [B, H_kv] (device
+ * float).  Arithmetic is fp32. */
+EA_API ea_status ea_router(const void* hidden, ea_dtype dtype, int B, int S, int D, int H_kv, int d,
+                    const ea_router_weights* weights, const ea_router_params* params,
+                    int32_t* head_mode, float* logits,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Hybrid-head attention (section 2 "Hybrid Head Mechanism"; section 3
+ * "Efficient Deployment"; appendix D.1 "Sparse Inference": the routing
+ * metadata goes straight into one kernel launch).
+ *   kind(b, h)  = head_mode[b, h] ? kind_if_sparse[h] : kind_if_dense[h]
+ *   o[b,i,h_q]  = sum_{j in L(i)} softmax_j(scale * q_i . k_j) v_j
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int n_sink;                   /* streaming sink tokens (>= 0); pages: 128        */
+  int window;                   /* streaming local window incl. the query (>= 1)   */
+  int block;                    /* block-sparse block edge; must be 128 here       */
+  const int32_t* bs_row_ptr;    /* device CSR [B*H_kv*ceil(S/block) + 1]; rows r = */
+  const int32_t* bs_col;        /*   (b*H_kv + h)*n_qb + qb; cols sorted, with qb  */
+  long long bs_nnz;             /* entries in bs_col (bounds every column read)    */
+  const int8_t* kind_if_dense;  /* host [H_kv]: ea_kind of a dense decision        */
+  const int8_t* kind_if_sparse; /* host [H_kv]: ea_kind of a sparse decision       */
+  float softmax_scale;          /* 0 selects 1/sqrt(d)                             */
+} ea_pattern_params;
+
+/* Bytes of workspace the attention calls and ea_effective_sparsity need. */
+EA_API size_t ea_attn_workspace_size(int B, int S, int H_q, int H_kv);
+
+/* One call = schedule build + attention launch (below).  dtype bf16: d == 128,
+ * tcgen05 tensor cores, fp32 softmax and accumulation, bf16 output.  dtype
+ * f32: d in {64, 128}, fp32 CUDA-core kernel (exact fp32 arithmetic).
+ * H_q % H_kv == 0, S >= 1.  head_mode: device int32 [B, H_kv]. */
+EA_API ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void* v, ea_dtype dtype,
+                                 int B, int S, int H_q, int H_kv, int d,
+                                 const int32_t* head_mode, const ea_pattern_params* pattern,
+                                 void* o, void* workspace, size_t workspace_bytes, void* stream);
+
+/* The two halves of ea_hybrid_attn_prefill, for callers that time or reuse
+ * them.  ea_build_schedule reads head_mode and the pattern on the device and
+ * writes the list of live (query tile, head group) work items, longest first,
+ * into the workspace; ea_attn_scheduled runs the attention kernel over that
+ * list and must receive the same head_mode, pattern and shapes. */
+EA_API ea_status ea_build_schedule(const int32_t* head_mode, const ea_pattern_params* pattern,
+                            int B, int S, int H_q, int H_kv, int d,
+                            void* workspace, size_t workspace_bytes, void* stream);
+EA_API ea_status ea_attn_scheduled(const void* q, const void* k, const void* v, ea_dtype dtype,
+                            int B, int S, int H_q, int H_kv, int d,
+                            const int32_t* head_mode, const ea_pattern_params* pattern,
+                            void* o, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Sparsity report (section 2 "Sparsity Ratio Computation"; appendix C.1).
+ * Omega_MSR per sample = sparse KV heads / H_kv.  Omega_ESR = 1 - live
+ * (query, key) pairs / causal pairs over all samples and query heads.  Tiles
+ * are 128 x 128; live_flops = 4 * d * 128^2 per live tile per query head.
+ * Counts run on the device; the call synchronises `stream` and fills the
+ * host outputs.  omega_msr_per_sample: host float [B] (may be NULL).
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  double omega_msr_mean;
+  double omega_esr;
+  long long live_pairs, causal_pairs;
+  long long live_tiles, causal_tiles;
+  double live_flops;
+} ea_sparsity_report;
+
+EA_API ea_status ea_effective_sparsity(const int32_t* head_mode, const ea_pattern_params* pattern,
+                                int B, int S, int H_q, int H_kv, int d,
+                                float* omega_msr_per_sample, ea_sparsity_report* report,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, reads and clears the workspace's device status
+ * word: EA_OK, EA_ERR_TIMEOUT or EA_ERR_BAD_LAYOUT. */
+EA_API ea_status ea_workspace_status(void* workspace, void* stream);
+
+/* Static text for a status code. */
+EA_API const char* ea_status_string(ea_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* EA_H_ */

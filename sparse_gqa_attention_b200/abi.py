@@ -1,0 +1,234 @@
+"""Python binding of the C ABI in include/ea.h (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and does no
+arithmetic of its own: it checks that tensors live on the GPU with the
+expected dtype and layout, passes their device pointers and the current CUDA
+stream to libea.so, and turns a non-zero ea_status into an ``EAError``.  There
+is no fallback: without the built library (or without a GPU) the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from ctypes import POINTER, Structure, c_double, c_float, c_int, c_longlong, c_size_t, c_void_p
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libea.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "ea.h")
+
+EA_OK, EA_ERR_INVALID_ARG, EA_ERR_UNSUPPORTED, EA_ERR_CUDA, EA_ERR_TIMEOUT, EA_ERR_BAD_LAYOUT = range(6)
+EA_DT_F32, EA_DT_BF16 = 0, 1
+EA_FULL, EA_STREAMING, EA_BLOCK_SPARSE = 0, 1, 2
+MAX_KV_HEADS = 64
+
+
+class EAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_lib().ea_status_string(status).decode()} (ea_status {status})")
+
+
+class RouterParams(Structure):
+    _fields_ = [("n_boundary", c_int)]
+
+
+class RouterWeights(Structure):
+    _fields_ = [(n, c_void_p) for n in ("w_k", "w_t1", "b_t1", "w_t2", "b_t2", "w_r1", "b_r1", "w_o", "b_o")]
+
+
+class PatternParams(Structure):
+    _fields_ = [("n_sink", c_int), ("window", c_int), ("block", c_int),
+                ("bs_row_ptr", c_void_p), ("bs_col", c_void_p), ("bs_nnz", c_longlong),
+                ("kind_if_dense", c_void_p), ("kind_if_sparse", c_void_p), ("softmax_scale", c_float)]
+
+
+class SparsityReport(Structure):
+    _fields_ = [("omega_msr_mean", c_double), ("omega_esr", c_double),
+                ("live_pairs", c_longlong), ("causal_pairs", c_longlong),
+                ("live_tiles", c_longlong), ("causal_tiles", c_longlong), ("live_flops", c_double)]
+
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built; run __graft_entry__.build() or "
+                               "python -m sparse_gqa_attention_b200.build")
+        lib = ctypes.CDLL(LIB_PATH)
+        st = c_int
+        lib.ea_status_string.restype = ctypes.c_char_p
+        lib.ea_status_string.argtypes = [c_int]
+        lib.ea_router_workspace_size.restype = c_size_t
+        lib.ea_router_workspace_size.argtypes = [c_int, c_int, c_int, c_int]
+        lib.ea_attn_workspace_size.restype = c_size_t
+        lib.ea_attn_workspace_size.argtypes = [c_int, c_int, c_int, c_int]
+        lib.ea_router.restype = st
+        lib.ea_router.argtypes = [c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
+                                  POINTER(RouterWeights), POINTER(RouterParams), c_void_p, c_void_p,
+                                  c_void_p, c_size_t, c_void_p]
+        attn = [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
+                c_void_p, POINTER(PatternParams), c_void_p, c_void_p, c_size_t, c_void_p]
+        lib.ea_hybrid_attn_prefill.restype = st
+        lib.ea_hybrid_attn_prefill.argtypes = attn
+        lib.ea_attn_scheduled.restype = st
+        lib.ea_attn_scheduled.argtypes = attn
+        lib.ea_build_schedule.restype = st
+        lib.ea_build_schedule.argtypes = [c_void_p, POINTER(PatternParams), c_int, c_int, c_int, c_int, c_int,
+                                          c_void_p, c_size_t, c_void_p]
+        lib.ea_effective_sparsity.restype = st
+        lib.ea_effective_sparsity.argtypes = [c_void_p, POINTER(PatternParams), c_int, c_int, c_int, c_int, c_int,
+                                              c_void_p, POINTER(SparsityReport), c_void_p, c_size_t, c_void_p]
+        lib.ea_workspace_status.restype = st
+        lib.ea_workspace_status.argtypes = [c_void_p, c_void_p]
+        _LIB = lib
+    return _LIB
+
+
+def declared_symbols():
+    """Names of the functions include/ea.h exports."""
+    text = open(HEADER_PATH).read()
+    return sorted(set(re.findall(r"EA_API\s+[\w\s\*]+?\b(ea_\w+)\s*\(", text)))
+
+
+def _check(status: int, where: str):
+    if status != EA_OK:
+        raise EAError(status, where)
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return c_void_p(s.cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (row-major)")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return c_void_p(t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return EA_DT_BF16
+    if t.dtype == torch.float32:
+        return EA_DT_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; bfloat16 or float32")
+
+
+class Pattern:
+    """Device-side block layout plus host kind tables, kept alive for the C struct."""
+
+    def __init__(self, n_sink, window, block, row_ptr, cols, kind_if_dense, kind_if_sparse,
+                 softmax_scale=0.0, device="cuda"):
+        self.n_sink, self.window, self.block = int(n_sink), int(window), int(block)
+        self.row_ptr = torch.as_tensor(np.asarray(row_ptr, np.int32)).to(device)
+        self.cols = torch.as_tensor(np.asarray(cols, np.int32)).to(device)
+        self.kind_if_dense = np.ascontiguousarray(kind_if_dense, dtype=np.int8)
+        self.kind_if_sparse = np.ascontiguousarray(kind_if_sparse, dtype=np.int8)
+        self.softmax_scale = float(softmax_scale)
+
+    @classmethod
+    def from_workloads(cls, p, device="cuda"):
+        return cls(p.n_sink, p.window, p.block, p.row_ptr, p.cols, p.kind_if_dense, p.kind_if_sparse,
+                   p.softmax_scale, device)
+
+    def c_struct(self) -> PatternParams:
+        return PatternParams(self.n_sink, self.window, self.block,
+                             c_void_p(self.row_ptr.data_ptr() if self.cols.numel() else 0),
+                             c_void_p(self.cols.data_ptr() if self.cols.numel() else 0),
+                             self.cols.numel(),
+                             self.kind_if_dense.ctypes.data_as(c_void_p),
+                             self.kind_if_sparse.ctypes.data_as(c_void_p),
+                             self.softmax_scale)
+
+
+# ---------------------------------------------------------------------------
+# Router
+# ---------------------------------------------------------------------------
+
+def ea_router_workspace_size(B: int, S: int, D: int, n_boundary: int = 100) -> int:
+    return int(_lib().ea_router_workspace_size(B, S, D, n_boundary))
+
+
+def ea_router(hidden: torch.Tensor, weights: dict, head_mode: torch.Tensor, workspace: torch.Tensor,
+              n_boundary: int = 100, logits: torch.Tensor | None = None, stream=None):
+    """head_mode[B, H_kv] (int32, device) <- router(hidden[B, S, D]); optional logits (float32)."""
+    B, S, D = hidden.shape
+    H_kv = weights["w_o"].shape[0]
+    d = weights["w_t1"].shape[1]
+    w = RouterWeights(*[_dev(weights[n], n) for n in
+                        ("w_k", "w_t1", "b_t1", "w_t2", "b_t2", "w_r1", "b_r1", "w_o", "b_o")])
+    prm = RouterParams(n_boundary)
+    status = _lib().ea_router(_dev(hidden, "hidden"), _dtype_code(hidden), B, S, D, H_kv, d, ctypes.byref(w),
+                              ctypes.byref(prm), _dev(head_mode, "head_mode", torch.int32),
+                              _dev(logits, "logits", torch.float32) if logits is not None else None,
+                              _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+                              _stream(stream))
+    _check(status, "ea_router")
+
+
+# ---------------------------------------------------------------------------
+# Hybrid attention
+# ---------------------------------------------------------------------------
+
+def ea_attn_workspace_size(B: int, S: int, H_q: int, H_kv: int) -> int:
+    return int(_lib().ea_attn_workspace_size(B, S, H_q, H_kv))
+
+
+def _attn_args(q, k, v, head_mode, pattern: Pattern, o, workspace, stream):
+    B, S, H_q, d = q.shape
+    H_kv = k.shape[2]
+    p = pattern.c_struct()
+    return (_dev(q, "q"), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype), _dtype_code(q), B, S, H_q, H_kv, d,
+            _dev(head_mode, "head_mode", torch.int32), ctypes.byref(p), _dev(o, "o", q.dtype),
+            _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream)), p
+
+
+def ea_hybrid_attn_prefill(q, k, v, head_mode, pattern: Pattern, o, workspace, stream=None):
+    """o[B, S, H_q, d] <- hybrid-head attention of q, k, v under head_mode and pattern."""
+    args, keep = _attn_args(q, k, v, head_mode, pattern, o, workspace, stream)
+    _check(_lib().ea_hybrid_attn_prefill(*args), "ea_hybrid_attn_prefill")
+
+
+def ea_build_schedule(head_mode, pattern: Pattern, B, S, H_q, H_kv, d, workspace, stream=None):
+    p = pattern.c_struct()
+    _check(_lib().ea_build_schedule(_dev(head_mode, "head_mode", torch.int32), ctypes.byref(p), B, S, H_q, H_kv,
+                                    d, _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+                                    _stream(stream)), "ea_build_schedule")
+
+
+def ea_attn_scheduled(q, k, v, head_mode, pattern: Pattern, o, workspace, stream=None):
+    args, keep = _attn_args(q, k, v, head_mode, pattern, o, workspace, stream)
+    _check(_lib().ea_attn_scheduled(*args), "ea_attn_scheduled")
+
+
+def ea_effective_sparsity(head_mode, pattern: Pattern, B, S, H_q, H_kv, d, workspace, stream=None):
+    """(Omega_MSR per sample [B] numpy, report dict); synchronises the stream."""
+    p = pattern.c_struct()
+    per = np.zeros(B, np.float32)
+    rep = SparsityReport()
+    status = _lib().ea_effective_sparsity(_dev(head_mode, "head_mode", torch.int32), ctypes.byref(p), B, S, H_q,
+                                          H_kv, d, per.ctypes.data_as(c_void_p), ctypes.byref(rep),
+                                          _dev(workspace, "workspace"),
+                                          workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(status, "ea_effective_sparsity")
+    return per, {f: getattr(rep, f) for f, _ in SparsityReport._fields_}
+
+
+def ea_workspace_status(workspace, stream=None) -> int:
+    """Reads and clears the workspace status word; returns the ea_status it maps to."""
+    return int(_lib().ea_workspace_status(_dev(workspace, "workspace"), _stream(stream)))
+
+
+def ea_status_string(status: int) -> str:
+    return _lib().ea_status_string(status).decode()

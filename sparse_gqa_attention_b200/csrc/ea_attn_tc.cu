@@ -1,0 +1,513 @@
+// ea_attn_tc.cu — hybrid-head GQA prefill attention on the sm_100a tensor cores.
+//
+// What it computes ("Elastic Attention: Test-time Adaptive Sparsity Ratios for
+// Efficient Transformers", section 2 "Hybrid Head Mechanism", section 3
+// "Attention Router" / "Efficient Deployment", appendix D.1 "Sparse Inference"):
+// every query head runs the pattern of its KV head's routed kind (full causal,
+// streaming sink + window, block-sparse) and its output goes to its own slot of
+// o[b, i, h_q, :]; all kinds run in this one launch, fed by the device-built
+// work list, and only the live key tiles of each head are visited.
+//
+// Design (B200): persistent CTAs, one per SM, walking the cost-sorted work list in
+// a snake order.  A work item is 128 query rows of two query heads of one KV
+// group (two "slots"), so every K/V tile brought into shared memory feeds two
+// 128x128 products.  Warp roles, 384 threads:
+//   warp 0      TMA producer: Q tiles of both slots, then K and V tiles of each
+//               live key tile into an NST-stage ring (128-byte swizzle, 2 boxes
+//               of 64 columns per 128x128 tile).  No cluster multicast.
+//   warp 1      TMEM owner and MMA issuer (one thread): S_s = Q_s K^T (SS MMA,
+//               M=N=128, K=16 steps) into TMEM, then O_s += P_s V (TS MMA: P
+//               read from TMEM, V from shared memory as an MN-major operand).
+//   warps 4-7   softmax for slot 0, warps 8-11 for slot 1: one thread per query
+//               row (its TMEM lane).  Reads S from TMEM, applies the element rule
+//               only on boundary tiles, keeps a running max that is raised only
+//               when a new maximum exceeds it by 2^8 (the stale max cancels in
+//               the final division), rescales O in TMEM when it is raised, writes
+//               P as bf16 over the S columns, and finally divides O by the row
+//               sum and stores bf16 rows.
+// TMEM: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512) fp32 columns; P_s
+// aliases the first 64 columns of S_s (bf16 pairs).  Before S_s is overwritten
+// by the next Q K^T product, the MMA thread waits for the P V product that reads
+// P_s: tcgen05 only orders MMAs on the same accumulator, so this keeps the P
+// reads ahead of the S writes by construction.
+// Every mbarrier wait is bounded (kWaitLimitNs); on expiry the CTA raises an
+// abort flag, records kStatusTimeout in the workspace status word, drains its
+// own copies and MMAs, frees TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <mutex>
+#include "ea_common.cuh"
+#include "ea_internal.h"
+#include "ea_sm100.cuh"
+
+namespace ea {
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128, BN = 128, HD = 128;
+constexpr int NST = 2;                                 // K/V stages
+constexpr int kThreads = 384;
+constexpr uint32_t kTileBytes = BM * HD * 2;           // 32 KB per 128x128 bf16 tile
+constexpr uint32_t kBoxBytes = kTileBytes / 2;         // one 64-column box
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_K = 2 * kTileBytes;
+constexpr uint32_t OFF_V = OFF_K + NST * kTileBytes;
+constexpr uint32_t OFF_BAR = OFF_V + NST * kTileBytes;
+enum : int {
+  B_QFULL = 0, B_QEMPTY = 2, B_KFULL = 4, B_VFULL = B_KFULL + NST, B_KVEMPTY = B_VFULL + NST,
+  B_SFULL = B_KVEMPTY + NST, B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2, B_OFULL = B_PVDONE + 2,
+  B_FIN = B_OFULL + 2, N_BAR = B_FIN + 1
+};
+constexpr uint32_t OFF_TMEM = OFF_BAR + N_BAR * 8;
+constexpr uint32_t OFF_ABORT = OFF_TMEM + 4;
+constexpr uint32_t kSmemBytes = OFF_ABORT + 4 + 1024;  // + slack to align the base to 1024
+constexpr uint32_t kTmemCols = 512;
+__device__ __forceinline__ uint32_t col_s(int s) { return 128u * s; }        // S_s (and P_s) columns
+__device__ __forceinline__ uint32_t col_o(int s) { return 256u + 128u * s; } // O_s columns
+constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, false);
+constexpr uint32_t IDESC_PV = idesc_bf16(BM, HD, true);
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr float kRescaleLog2 = 8.0f;
+// Register split: the launch gives 384 x 168 = 64512 registers; warpgroup 0 (producer,
+// MMA, two idle warps) drops to 88 and the two softmax warpgroups rise to 208:
+// 128 x 88 + 256 x 208 = 64512.
+constexpr int kRegsCtl = 88, kRegsSoftmax = 208;
+static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= kThreads * 168, "register split exceeds the launch");
+
+struct Ctx {
+  uint32_t bar0;                 // shared address of barrier 0
+  volatile int* abort_flag;
+  uint32_t* status;
+  __device__ uint32_t bar(int i) const { return bar0 + 8u * i; }
+};
+
+__device__ __forceinline__ bool wait_slow(const Ctx& c, uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*c.abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *c.abort_flag = 1;
+      atomicOr(c.status, kStatusTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ bool wait(const Ctx& c, uint32_t bar, uint32_t parity) {
+  return mbar_try_wait(bar, parity) || wait_slow(c, bar, parity);
+}
+
+struct Item {
+  int b, h, t, pr, kind, n, sink_end, win_lo;
+  long long csr_beg;
+  bool two;
+};
+
+__device__ __forceinline__ int item_index(int it, int cta, int ncta) {
+  return it * ncta + ((it & 1) ? (ncta - 1 - cta) : cta);
+}
+
+__device__ __forceinline__ Item load_item(const int4* items, int idx, const PatternDev& p,
+                                          const int32_t* head_mode, int H_kv, int G) {
+  const int4 w = items[idx];
+  Item I;
+  I.b = w.x; I.h = w.y; I.t = w.z; I.pr = w.w;
+  I.kind = head_kind(p, head_mode, H_kv, I.b, I.h);
+  I.two = 2 * I.pr + 1 < G;
+  I.sink_end = I.win_lo = 0;
+  I.csr_beg = 0;
+  if (I.kind == EA_STREAMING) {
+    stream_ranges(p, I.t, I.sink_end, I.win_lo);
+    I.n = I.sink_end + max(0, I.t - I.win_lo + 1);
+  } else if (I.kind == EA_BLOCK_SPARSE) {
+    long long a, e;
+    csr_row(p, H_kv, I.b, I.h, I.t, a, e);
+    I.csr_beg = a;
+    I.n = (int)(e - a);
+  } else {
+    I.n = I.t + 1;
+  }
+  return I;
+}
+
+__device__ __forceinline__ uint64_t qk_desc(uint32_t tile, int kk) {
+  // K-major operand: rows of 128 bytes, 8-row swizzle atoms 1024 bytes apart (SBO);
+  // K step kk of 16 elements = +32 bytes inside a 64-column box, boxes 16 KB apart.
+  return sdesc_sw128(tile + (uint32_t)(kk >> 2) * kBoxBytes + (uint32_t)(kk & 3) * 32u, 16u, 1024u);
+}
+__device__ __forceinline__ uint64_t v_desc(uint32_t tile, int kk) {
+  // MN-major operand (N = head dim, contiguous): 64-column boxes 16 KB apart (LBO),
+  // 8-key groups 1024 bytes apart (SBO); K step kk of 16 keys = +2048 bytes.
+  return sdesc_sw128(tile + (uint32_t)kk * 2048u, kBoxBytes, 1024u);
+}
+
+// S_s = Q_s K^T for the key tile in stage st.  With kSafeAlias the previous P_s V
+// product (which reads P_s inside the S_s columns) is complete before S_s is written.
+template <bool kSafeAlias>
+__device__ __forceinline__ bool issue_qk(const Ctx& c, uint32_t tmem, uint32_t base, int s, int st, bool& pend,
+                                         int pv_cnt) {
+  if (kSafeAlias && pend) {
+    if (!wait(c, c.bar(B_PVDONE + s), (pv_cnt - 1) & 1)) return false;
+    pend = false;
+  }
+  fence_after_sync();
+  const uint32_t qt = base + OFF_Q + s * kTileBytes, kt = base + OFF_K + st * kTileBytes;
+#pragma unroll
+  for (int kk = 0; kk < HD / 16; ++kk)
+    mma_ss(tmem + col_s(s), qk_desc(qt, kk), qk_desc(kt, kk), IDESC_QK, kk > 0 ? 1u : 0u);
+  commit(c.bar(B_SFULL + s));
+  return true;
+}
+
+// O_s (+)= P_s V for the key tile in stage st, once the softmax has written P_s.
+__device__ __forceinline__ bool issue_pv(const Ctx& c, uint32_t tmem, uint32_t base, int s, int st, bool accumulate,
+                                         bool last, int& p_cnt, int& pv_cnt, bool& pend) {
+  if (!wait(c, c.bar(B_PFULL + s), p_cnt & 1)) return false;
+  ++p_cnt;
+  fence_after_sync();
+  const uint32_t vt = base + OFF_V + st * kTileBytes;
+#pragma unroll
+  for (int kk = 0; kk < BN / 16; ++kk)
+    mma_ts(tmem + col_o(s), tmem + col_s(s) + 8u * kk, v_desc(vt, kk), IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
+  commit(c.bar(B_PVDONE + s));
+  ++pv_cnt;
+  pend = true;
+  if (last) {
+    commit(c.bar(B_OFULL + s));
+    commit(c.bar(B_QEMPTY + s));
+  }
+  return true;
+}
+
+// One 128-key tile of one query row: running max (raised only past kRescaleLog2),
+// row sum, and P = exp2(scale*log2e*s - max) stored as bf16 pairs over the first 64
+// S columns at p_addr.  kMode 0: every key live; 1: causal rule; 2: streaming rule.
+// Returns the factor O must be multiplied by (1 when the max was not raised).
+template <int kMode>
+__device__ __forceinline__ float softmax_tile(const float (&x)[BN], int lim, int sink_lim, int win_lim,
+                                              float scale_log2, float& m_ref, float& l, uint32_t p_addr) {
+  auto live = [&](int e) {
+    if (kMode == 0) return true;
+    if (kMode == 1) return e <= lim;
+    return e <= lim && (e < sink_lim || e > win_lim);
+  };
+  float mt = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < BN; ++e) mt = fmaxf(mt, live(e) ? x[e] : -INFINITY);
+  const float mts = mt * scale_log2;
+  float f = 1.f;
+  if (mts > m_ref + kRescaleLog2) {
+    f = ex2(m_ref - mts);  // 0 while m_ref is still -inf
+    l *= f;
+    m_ref = mts;
+  }
+  const float sub = (m_ref == -INFINITY) ? 0.f : m_ref;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int e = 0; e < 64; e += 2) {
+      const int e0 = 64 * half + e;
+      const float p0 = live(e0) ? ex2(fmaf(x[e0], scale_log2, -sub)) : 0.f;
+      const float p1 = live(e0 + 1) ? ex2(fmaf(x[e0 + 1], scale_log2, -sub)) : 0.f;
+      l += p0 + p1;
+      pk[e / 2] = pack_bf16x2(p0, p1);
+    }
+    tmem_st32(p_addr + 32 * half, pk);
+  }
+  return f;
+}
+
+template <bool kSafeAlias>
+__global__ void __launch_bounds__(kThreads, 1)
+hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o,
+                      const int32_t* __restrict__ head_mode, const PatternDev p, int S, int H_q, int H_kv,
+                      const int4* __restrict__ items, uint32_t* __restrict__ hdr) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int G = H_q / H_kv;
+  Ctx c;
+  c.bar0 = base + OFF_BAR;
+  c.abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_ABORT);
+  c.status = hdr + kWsStatus / 4;
+  const int n_items = (int)hdr[kWsNItems / 4];
+
+  if (threadIdx.x == 0) {
+    tma_prefetch_map(&tm_q);
+    tma_prefetch_map(&tm_k);
+    tma_prefetch_map(&tm_v);
+    for (int i = 0; i < N_BAR; ++i) {
+      const bool softmax_arrive = (i == B_PFULL || i == B_PFULL + 1);
+      mbar_init(c.bar(i), softmax_arrive ? 128u : 1u);
+    }
+    *c.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(base + OFF_TMEM, kTmemCols);
+    tmem_relinquish();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + OFF_TMEM);
+  if (warp < 4) regs_dec<kRegsCtl>();
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int q_use[2] = {0, 0};
+      int kv_it = 0;
+      bool ok = true;
+      for (int it = 0; ok; ++it) {
+        const int idx = item_index(it, blockIdx.x, gridDim.x);
+        if (idx >= n_items) break;
+        const Item I = load_item(items, idx, p, head_mode, H_kv, G);
+        if (I.n == 0) continue;
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+          if (!ok || (s == 1 && !I.two)) continue;
+          ok = wait(c, c.bar(B_QEMPTY + s), (q_use[s] & 1) ^ 1);
+          if (!ok) continue;
+          const int h_q = I.h * G + 2 * I.pr + s;
+          const uint32_t dst = base + OFF_Q + s * kTileBytes;
+          mbar_expect_tx(c.bar(B_QFULL + s), kTileBytes);
+          tma_load_4d(dst, &tm_q, c.bar(B_QFULL + s), 0, h_q, I.t * BM, I.b);
+          tma_load_4d(dst + kBoxBytes, &tm_q, c.bar(B_QFULL + s), 64, h_q, I.t * BM, I.b);
+          ++q_use[s];
+        }
+        for (int jj = 0; jj < I.n && ok; ++jj) {
+          const int ct = max(0, live_tile(p, I.kind, I.t, jj, I.sink_end, I.win_lo, I.csr_beg));
+          const int st = kv_it % NST;
+          ok = wait(c, c.bar(B_KVEMPTY + st), ((kv_it / NST) & 1) ^ 1);
+          if (!ok) break;
+          const uint32_t kdst = base + OFF_K + st * kTileBytes, vdst = base + OFF_V + st * kTileBytes;
+          mbar_expect_tx(c.bar(B_KFULL + st), kTileBytes);
+          tma_load_4d(kdst, &tm_k, c.bar(B_KFULL + st), 0, I.h, ct * BN, I.b);
+          tma_load_4d(kdst + kBoxBytes, &tm_k, c.bar(B_KFULL + st), 64, I.h, ct * BN, I.b);
+          mbar_expect_tx(c.bar(B_VFULL + st), kTileBytes);
+          tma_load_4d(vdst, &tm_v, c.bar(B_VFULL + st), 0, I.h, ct * BN, I.b);
+          tma_load_4d(vdst + kBoxBytes, &tm_v, c.bar(B_VFULL + st), 64, I.h, ct * BN, I.b);
+          ++kv_it;
+        }
+      }
+      // Drain: the last copy armed on every barrier has landed before the CTA exits.
+      for (int st = 0; st < NST; ++st) {
+        const int uses = kv_it / NST + (st < kv_it % NST ? 1 : 0);
+        if (uses > 0) {
+          wait_slow(c, c.bar(B_KFULL + st), (uses - 1) & 1);
+          wait_slow(c, c.bar(B_VFULL + st), (uses - 1) & 1);
+        }
+      }
+#pragma unroll
+      for (int s = 0; s < 2; ++s)
+        if (q_use[s] > 0) wait_slow(c, c.bar(B_QFULL + s), (q_use[s] - 1) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int q_use0 = 0, q_use1 = 0, p_cnt0 = 0, p_cnt1 = 0, pv_cnt0 = 0, pv_cnt1 = 0;
+      bool pend0 = false, pend1 = false;
+      int kv_it = 0;
+      bool ok = true;
+      for (int it = 0; ok; ++it) {
+        const int idx = item_index(it, blockIdx.x, gridDim.x);
+        if (idx >= n_items) break;
+        const Item I = load_item(items, idx, p, head_mode, H_kv, G);
+        if (I.n == 0) continue;
+        ok = wait(c, c.bar(B_QFULL + 0), q_use0 & 1);
+        ++q_use0;
+        if (I.two) {
+          ok = ok && wait(c, c.bar(B_QFULL + 1), q_use1 & 1);
+          ++q_use1;
+        }
+        ok = ok && wait(c, c.bar(B_KFULL + kv_it % NST), (kv_it / NST) & 1);
+        if (ok) {
+          ok = issue_qk<kSafeAlias>(c, tmem, base, 0, kv_it % NST, pend0, pv_cnt0);
+          if (ok && I.two) ok = issue_qk<kSafeAlias>(c, tmem, base, 1, kv_it % NST, pend1, pv_cnt1);
+        }
+        for (int jj = 0; jj < I.n && ok; ++jj) {
+          const int st = kv_it % NST, st1 = (kv_it + 1) % NST;
+          const bool last = jj + 1 == I.n;
+          ok = wait(c, c.bar(B_VFULL + st), (kv_it / NST) & 1);
+          if (ok) ok = issue_pv(c, tmem, base, 0, st, jj > 0, last, p_cnt0, pv_cnt0, pend0);
+          if (ok && !last) {
+            ok = wait(c, c.bar(B_KFULL + st1), ((kv_it + 1) / NST) & 1);
+            if (ok) ok = issue_qk<kSafeAlias>(c, tmem, base, 0, st1, pend0, pv_cnt0);
+          }
+          if (ok && I.two) {
+            ok = issue_pv(c, tmem, base, 1, st, jj > 0, last, p_cnt1, pv_cnt1, pend1);
+            if (ok && !last) ok = issue_qk<kSafeAlias>(c, tmem, base, 1, st1, pend1, pv_cnt1);
+          }
+          commit(c.bar(B_KVEMPTY + st));
+          ++kv_it;
+        }
+      }
+      commit(c.bar(B_FIN));                       // every MMA issued here has completed
+      wait_slow(c, c.bar(B_FIN), 0);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax slots
+    regs_inc<kRegsSoftmax>();
+    const int s = (warp - 4) / 4;
+    const int row = (warp % 4) * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
+    int s_cnt = 0, o_cnt = 0;
+    bool ok = true;
+    for (int it = 0; ok; ++it) {
+      const int idx = item_index(it, blockIdx.x, gridDim.x);
+      if (idx >= n_items) break;
+      const Item I = load_item(items, idx, p, head_mode, H_kv, G);
+      if (I.n == 0 || (s == 1 && !I.two)) continue;
+      const int i = I.t * BM + row;
+      const int kind_el = I.kind == EA_STREAMING ? EA_STREAMING : EA_FULL;
+      float m_ref = -INFINITY, l = 0.f;
+      for (int jj = 0; jj < I.n; ++jj) {
+        const int ct = live_tile(p, I.kind, I.t, jj, I.sink_end, I.win_lo, I.csr_beg);
+        ok = wait(c, c.bar(B_SFULL + s), s_cnt & 1);
+        ++s_cnt;
+        if (!ok) break;
+        fence_after_sync();
+        float x[BN];
+        {
+          uint32_t r[BN];
+#pragma unroll
+          for (int q4 = 0; q4 < BN / 32; ++q4) tmem_ld32(lane_addr + col_s(s) + 32 * q4, r + 32 * q4);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < BN; ++e) x[e] = __uint_as_float(r[e]);
+        }
+        // Key j = 128*ct + e is live iff e <= lim (causal) and, for a streaming head,
+        // e < sink_lim or e > win_lim.  Unmasked tiles skip the test.
+        float f;
+        if (ct < 0) {
+          f = softmax_tile<1>(x, -1, 0, 0, p.scale_log2, m_ref, l, lane_addr + col_s(s));
+        } else if (tile_needs_mask(p, I.kind, I.t, ct)) {
+          const int lim = i - ct * BN;
+          if (kind_el == EA_STREAMING)
+            f = softmax_tile<2>(x, lim, p.n_sink - ct * BN, lim - p.window, p.scale_log2, m_ref, l,
+                                lane_addr + col_s(s));
+          else
+            f = softmax_tile<1>(x, lim, 0, 0, p.scale_log2, m_ref, l, lane_addr + col_s(s));
+        } else {
+          f = softmax_tile<0>(x, 0, 0, 0, p.scale_log2, m_ref, l, lane_addr + col_s(s));
+        }
+        const bool raise = f != 1.f;
+        if (jj > 0 && __any_sync(0xffffffffu, raise)) {   // O (complete up to tile jj-1) *= f
+#pragma unroll 1
+          for (int q4 = 0; q4 < HD / 32; ++q4) {
+            uint32_t r[32];
+            tmem_ld32(lane_addr + col_o(s) + 32 * q4, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
+            tmem_st32(lane_addr + col_o(s) + 32 * q4, r);
+          }
+        }
+        tmem_st_wait();
+        fence_before_sync();
+        mbar_arrive(c.bar(B_PFULL + s));
+      }
+      if (!ok) break;
+      ok = wait(c, c.bar(B_OFULL + s), o_cnt & 1);
+      ++o_cnt;
+      if (!ok) break;
+      fence_after_sync();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const int h_q = I.h * G + 2 * I.pr + s;
+      __nv_bfloat16* orow = o + (((size_t)I.b * S + i) * H_q + h_q) * HD;
+#pragma unroll
+      for (int q4 = 0; q4 < HD / 32; ++q4) {
+        uint32_t r[32];
+        tmem_ld32(lane_addr + col_o(s) + 32 * q4, r);
+        tmem_ld_wait();
+        if (i < S) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(r[e]) * inv, __uint_as_float(r[e + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(r[e + 2]) * inv, __uint_as_float(r[e + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(r[e + 4]) * inv, __uint_as_float(r[e + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(r[e + 6]) * inv, __uint_as_float(r[e + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + 32 * q4 + e) = w;
+          }
+        }
+      }
+      fence_before_sync();
+    }
+  }
+
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// [B, S, H, 128] bf16 viewed as 4-D (d, H, S, B); box = 64 columns x 1 head x 128 rows.
+bool make_map(CUtensorMap* m, const void* ptr, int B, int S, int H) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)HD * 2, (cuuint64_t)H * HD * 2, (cuuint64_t)S * H * HD * 2};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)BM, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+}  // namespace
+
+ea_status launch_attn_tc(const void* q, const void* k, const void* v, void* o, const int32_t* head_mode,
+                         const PatternDev& pat, int B, int S, int H_q, int H_kv, void* workspace,
+                         cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, B, S, H_q) || !make_map(&mk, k, B, S, H_kv) || !make_map(&mv, v, B, S, H_kv))
+    return EA_ERR_CUDA;
+  const long long n_items = (long long)B * H_kv * pat.n_qt * n_pairs(H_q, H_kv);
+  const int grid = (int)std::min<long long>(n_items, sm_count());
+  auto kern = hybrid_attn_tc_kernel<true>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) != cudaSuccess)
+    return EA_ERR_CUDA;
+  char* ws = static_cast<char*>(workspace);
+  const size_t items_off = kWsHeader + ((size_t)B * 4 + 255) / 256 * 256;
+  kern<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), head_mode, pat, S, H_q,
+                                           H_kv, reinterpret_cast<const int4*>(ws + items_off),
+                                           reinterpret_cast<uint32_t*>(ws));
+  return cudaGetLastError() == cudaSuccess ? EA_OK : EA_ERR_CUDA;
+}
+
+}  // namespace ea

@@ -1,0 +1,118 @@
+// ea_common.cuh — device-side definitions shared by the schedule builder, the
+// attention kernels and the sparsity counter.
+//
+// Live key tiles per head kind, for a 128-row query tile t (rows 128t..128t+127)
+// and 128-key tiles c (keys 128c..128c+127); the element rules follow section 2
+// "Hybrid Head Mechanism" and appendix D.1 "Sparse Inference" of "Elastic
+// Attention: Test-time Adaptive Sparsity Ratios for Efficient Transformers":
+//   FULL          tiles 0..t; only the diagonal tile t needs the causal mask.
+//   STREAMING     sink tiles 0..ceil(n_sink/128)-1 (at most t), then window tiles
+//                 floor(max(0, 128t - window + 1)/128)..t (not repeating sink tiles).
+//                 Every enumerated tile holds at least one live pair.
+//   BLOCK_SPARSE  (block == 128) the listed key blocks of CSR row
+//                 (b*H_kv + h)*n_qt + t; the diagonal tile needs the causal mask.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+#include "../../include/ea.h"
+
+namespace ea {
+
+constexpr int kTile = 128;
+
+// Workspace layout of the attention calls (bytes from the workspace base).
+constexpr size_t kWsStatus = 0;        // uint32 sticky status bits
+constexpr size_t kWsNItems = 4;        // uint32 items in the schedule
+constexpr size_t kWsLivePairs = 16;    // uint64
+constexpr size_t kWsLiveTiles = 24;    // uint64
+constexpr size_t kWsHeader = 256;
+// then int32 sparse-head count per sample, padded to 256 bytes, then int4 items.
+
+// Device status bits.
+constexpr uint32_t kStatusTimeout = 1u << 0;
+constexpr uint32_t kStatusBadLayout = 1u << 1;
+constexpr uint32_t kStatusBadMode = 1u << 2;
+
+struct PatternDev {
+  int n_sink;
+  int window;
+  int block;
+  int n_qt;                 // ceil(S / 128)
+  const int32_t* row_ptr;
+  const int32_t* cols;
+  long long nnz;
+  float scale;              // softmax scale
+  float scale_log2;         // softmax scale * log2(e)
+  int8_t kind_dense[EA_MAX_KV_HEADS];
+  int8_t kind_sparse[EA_MAX_KV_HEADS];
+};
+
+__host__ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+__device__ __forceinline__ int head_kind(const PatternDev& p, const int32_t* head_mode, int H_kv,
+                                         int b, int h) {
+  return head_mode[b * H_kv + h] != 0 ? p.kind_sparse[h] : p.kind_dense[h];
+}
+
+// Streaming tile ranges of query tile t: [0, sink_end) and [win_lo, t].
+__device__ __forceinline__ void stream_ranges(const PatternDev& p, int t, int& sink_end, int& win_lo) {
+  sink_end = min(cdiv(p.n_sink, kTile), t + 1);
+  int lo = max(0, t * kTile - p.window + 1) / kTile;
+  win_lo = max(lo, sink_end);
+}
+
+// CSR row [beg, end) of (b, h, t), clamped so a malformed row never reads outside bs_col.
+__device__ __forceinline__ void csr_row(const PatternDev& p, int H_kv, int b, int h, int t,
+                                        long long& beg, long long& end) {
+  long long r = ((long long)b * H_kv + h) * p.n_qt + t;
+  long long a = p.row_ptr[r], e = p.row_ptr[r + 1];
+  a = max(0LL, min(a, p.nnz));
+  e = max(a, min(e, p.nnz));
+  beg = a;
+  end = e;
+}
+
+// Number of live key tiles of query tile t.
+__device__ __forceinline__ int n_live_tiles(const PatternDev& p, int kind, int H_kv, int b, int h, int t) {
+  if (kind == EA_STREAMING) {
+    int se, wl;
+    stream_ranges(p, t, se, wl);
+    return se + max(0, t - wl + 1);
+  }
+  if (kind == EA_BLOCK_SPARSE) {
+    long long a, e;
+    csr_row(p, H_kv, b, h, t, a, e);
+    return (int)(e - a);
+  }
+  return t + 1;
+}
+
+// Key tile index of the jj-th live tile (0 <= jj < n_live_tiles).  For block-sparse
+// heads a listed column outside [0, t] (a malformed layout) maps to -1: skip it.
+__device__ __forceinline__ int live_tile(const PatternDev& p, int kind, int t, int jj,
+                                         int sink_end, int win_lo, long long csr_beg) {
+  if (kind == EA_STREAMING) return jj < sink_end ? jj : win_lo + (jj - sink_end);
+  if (kind == EA_BLOCK_SPARSE) {
+    int c = p.cols[csr_beg + jj];
+    return (c >= 0 && c <= t) ? c : -1;
+  }
+  return jj;
+}
+
+// True when some pair of (query tile t, key tile c) may be dead, so the element rule
+// must run; false when every pair with a real query row is live.
+__device__ __forceinline__ bool tile_needs_mask(const PatternDev& p, int kind, int t, int c) {
+  if (c >= t) return true;                              // diagonal (causal) tile
+  if (kind != EA_STREAMING) return false;
+  if (c * kTile + kTile - 1 < p.n_sink) return false;   // all sink keys
+  return (t * kTile + kTile - 1) - c * kTile >= p.window;
+}
+
+// Element rule: is key j live for query row i.
+__device__ __forceinline__ bool key_live(const PatternDev& p, int kind, int i, int j) {
+  if (j > i) return false;
+  if (kind == EA_STREAMING) return j < p.n_sink || i - j < p.window;
+  return true;  // FULL, and BLOCK_SPARSE inside a listed tile (block == tile)
+}
+
+}  // namespace ea

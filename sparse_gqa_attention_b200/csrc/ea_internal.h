@@ -1,0 +1,27 @@
+// ea_internal.h — launchers behind the C ABI (host side, not exported).
+#pragma once
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+#include "../../include/ea.h"
+
+namespace ea {
+struct PatternDev;
+
+size_t router_workspace_bytes(int B, int S, int D, int n_boundary);
+ea_status launch_router(const void* hidden, ea_dtype dtype, int B, int S, int D, int H_kv, int d,
+                        const ea_router_weights* w, const ea_router_params* prm, int32_t* head_mode,
+                        float* logits, void* workspace, cudaStream_t st);
+
+size_t attn_workspace_bytes(int B, int S, int H_q, int H_kv);
+int n_pairs(int H_q, int H_kv);
+ea_status launch_schedule(const int32_t* head_mode, const PatternDev& pat, int B, int S, int H_q, int H_kv,
+                          void* workspace, cudaStream_t st);
+ea_status launch_sparsity(const int32_t* head_mode, const PatternDev& pat, int B, int S, int H_q, int H_kv,
+                          void* workspace, cudaStream_t st);
+ea_status launch_attn_simt(const float* q, const float* k, const float* v, float* o, const int32_t* head_mode,
+                           const PatternDev& pat, int B, int S, int H_q, int H_kv, int d, cudaStream_t st);
+ea_status launch_attn_tc(const void* q, const void* k, const void* v, void* o, const int32_t* head_mode,
+                         const PatternDev& pat, int B, int S, int H_q, int H_kv, void* workspace,
+                         cudaStream_t st);
+}  // namespace ea

@@ -1,0 +1,183 @@
+// ea_schedule.cu — device-side work list for the hybrid attention launch, and the
+// sparsity counters.
+//
+// The routing metadata (head_mode plus the per-head patterns) is turned into the
+// list of live work items on the device, with no host round trip, so that one
+// attention launch serves every head kind ("Elastic Attention: Test-time Adaptive
+// Sparsity Ratios for Efficient Transformers", appendix D.1 "Sparse Inference":
+// one unified launch fed by the routing metadata; section 3 "Efficient
+// Deployment").  A work item is (b, h_kv, query tile t, head pair): the pair is
+// query heads 2p and 2p+1 of the KV group, which read the same key tiles.  Items
+// are sorted by cost (live tiles x heads), longest first.
+//
+// The sparsity counters follow section 2 "Sparsity Ratio Computation": sparse
+// heads per sample (Omega_MSR), live query-key pairs and live 128x128 tiles.
+#include <cuda_runtime.h>
+#include <cstdint>
+#include "ea_common.cuh"
+#include "ea_internal.h"
+
+namespace ea {
+namespace {
+
+constexpr int kSchedThreads = 1024;
+constexpr int kMaxBins = 8192;
+
+__device__ __forceinline__ void decode_item(int x, int np, int n_qt, int H_kv, int& b, int& h, int& t, int& pr) {
+  pr = x % np;
+  int r = x / np;
+  t = r % n_qt;
+  r /= n_qt;
+  h = r % H_kv;
+  b = r / H_kv;
+}
+
+__device__ __forceinline__ int item_cost(const PatternDev& p, const int32_t* head_mode, int H_kv, int G,
+                                         int b, int h, int t, int pr, int n_bins) {
+  const int kind = head_kind(p, head_mode, H_kv, b, h);
+  const int n = n_live_tiles(p, kind, H_kv, b, h, t);
+  const int heads = min(2, G - 2 * pr);
+  return min(n * heads, n_bins - 1);
+}
+
+__global__ void __launch_bounds__(kSchedThreads)
+schedule_kernel(const int32_t* __restrict__ head_mode, PatternDev p, int H_kv, int G, int np, int n_items,
+                int n_bins, uint32_t* __restrict__ hdr, int4* __restrict__ items) {
+  __shared__ int bins[kMaxBins];
+  __shared__ int part[kSchedThreads];
+  const int tid = threadIdx.x;
+  for (int i = tid; i < n_bins; i += kSchedThreads) bins[i] = 0;
+  __syncthreads();
+  uint32_t bad = 0;
+  for (int x = tid; x < n_items; x += kSchedThreads) {
+    int b, h, t, pr;
+    decode_item(x, np, p.n_qt, H_kv, b, h, t, pr);
+    const int m = head_mode[b * H_kv + h];
+    if (m != 0 && m != 1) bad |= kStatusBadMode;
+    const int kind = head_kind(p, head_mode, H_kv, b, h);
+    if (kind == EA_BLOCK_SPARSE && pr == 0) {
+      const long long r = ((long long)b * H_kv + h) * p.n_qt + t;
+      const long long a0 = p.row_ptr[r], a1 = p.row_ptr[r + 1];
+      if (a0 < 0 || a1 < a0 || a1 > p.nnz || a1 == a0) {
+        bad |= kStatusBadLayout;
+      } else {
+        int prev = -1;
+        for (long long e = a0; e < a1; ++e) {
+          const int c = p.cols[e];
+          if (c <= prev || c > t) bad |= kStatusBadLayout;
+          prev = c;
+        }
+        if (prev != t) bad |= kStatusBadLayout;
+      }
+    }
+    atomicAdd(&bins[item_cost(p, head_mode, H_kv, G, b, h, t, pr, n_bins)], 1);
+  }
+  if (bad) atomicOr(hdr + kWsStatus / 4, bad);
+  __syncthreads();
+  // Exclusive scan of the bins in descending cost order: bins[c] <- items costing more than c.
+  const int chunk = (n_bins + kSchedThreads - 1) / kSchedThreads;
+  const int q0 = tid * chunk;  // descending position q <-> bin n_bins - 1 - q
+  int local = 0;
+  for (int q = q0; q < min(q0 + chunk, n_bins); ++q) local += bins[n_bins - 1 - q];
+  part[tid] = local;
+  __syncthreads();
+  for (int off = 1; off < kSchedThreads; off <<= 1) {  // Hillis-Steele inclusive scan
+    const int v = tid >= off ? part[tid - off] : 0;
+    __syncthreads();
+    part[tid] += v;
+    __syncthreads();
+  }
+  int run = part[tid] - local;
+  for (int q = q0; q < min(q0 + chunk, n_bins); ++q) {
+    const int c = n_bins - 1 - q;
+    const int cnt = bins[c];
+    bins[c] = run;
+    run += cnt;
+  }
+  __syncthreads();
+  for (int x = tid; x < n_items; x += kSchedThreads) {
+    int b, h, t, pr;
+    decode_item(x, np, p.n_qt, H_kv, b, h, t, pr);
+    const int pos = atomicAdd(&bins[item_cost(p, head_mode, H_kv, G, b, h, t, pr, n_bins)], 1);
+    items[pos] = make_int4(b, h, t, pr);
+  }
+  if (tid == 0) hdr[kWsNItems / 4] = (uint32_t)n_items;
+}
+
+// grid (n_qt, H_kv, B), 128 threads: thread = query row of tile t.
+__global__ void __launch_bounds__(kTile)
+sparsity_kernel(const int32_t* __restrict__ head_mode, PatternDev p, int S, int H_kv, int G,
+                unsigned long long* __restrict__ counters, int* __restrict__ sparse_heads) {
+  const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int i = t * kTile + threadIdx.x;
+  const int kind = head_kind(p, head_mode, H_kv, b, h);
+  long long cnt = 0;
+  if (i < S) {
+    if (kind == EA_STREAMING) {
+      cnt = min(i + 1, p.window) + max(0, min(p.n_sink, i - p.window + 1));
+    } else if (kind == EA_BLOCK_SPARSE) {
+      long long a, e;
+      csr_row(p, H_kv, b, h, t, a, e);
+      int below = 0;
+      bool diag = false;
+      for (long long x = a; x < e; ++x) {
+        const int c = p.cols[x];
+        below += (c >= 0 && c < t);
+        diag |= (c == t);
+      }
+      cnt = (long long)below * kTile + (diag ? (i - t * kTile + 1) : 0);
+    } else {
+      cnt = i + 1;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  __shared__ long long red[kTile / 32];
+  if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = cnt;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long s = 0;
+    for (int w = 0; w < kTile / 32; ++w) s += red[w];
+    atomicAdd(counters + 0, (unsigned long long)(s * G));
+    atomicAdd(counters + 1, (unsigned long long)n_live_tiles(p, kind, H_kv, b, h, t) * G);
+    if (t == 0 && head_mode[b * H_kv + h] != 0) atomicAdd(sparse_heads + b, 1);
+  }
+}
+
+}  // namespace
+
+int n_pairs(int H_q, int H_kv) { return (H_q / H_kv + 1) / 2; }
+
+static size_t items_offset(int B) { return kWsHeader + ((size_t)B * 4 + 255) / 256 * 256; }
+
+size_t attn_workspace_bytes(int B, int S, int H_q, int H_kv) {
+  const size_t n_items = (size_t)B * H_kv * cdiv(S, kTile) * n_pairs(H_q, H_kv);
+  return items_offset(B) + n_items * sizeof(int4);
+}
+
+ea_status launch_schedule(const int32_t* head_mode, const PatternDev& pat, int B, int S, int H_q, int H_kv,
+                          void* workspace, cudaStream_t st) {
+  const int G = H_q / H_kv, np = n_pairs(H_q, H_kv);
+  const long long n_items = (long long)B * H_kv * pat.n_qt * np;
+  if (n_items > (1LL << 30)) return EA_ERR_UNSUPPORTED;
+  const int n_bins = min(kMaxBins, 2 * pat.n_qt + 1);
+  char* ws = static_cast<char*>(workspace);
+  schedule_kernel<<<1, kSchedThreads, 0, st>>>(head_mode, pat, H_kv, G, np, (int)n_items, n_bins,
+                                               reinterpret_cast<uint32_t*>(ws),
+                                               reinterpret_cast<int4*>(ws + items_offset(B)));
+  return cudaGetLastError() == cudaSuccess ? EA_OK : EA_ERR_CUDA;
+}
+
+ea_status launch_sparsity(const int32_t* head_mode, const PatternDev& pat, int B, int S, int H_q, int H_kv,
+                          void* workspace, cudaStream_t st) {
+  char* ws = static_cast<char*>(workspace);
+  if (cudaMemsetAsync(ws + kWsLivePairs, 0, 16, st) != cudaSuccess) return EA_ERR_CUDA;
+  if (cudaMemsetAsync(ws + kWsHeader, 0, (size_t)B * 4, st) != cudaSuccess) return EA_ERR_CUDA;
+  dim3 grid(pat.n_qt, H_kv, B);
+  sparsity_kernel<<<grid, kTile, 0, st>>>(head_mode, pat, S, H_kv, H_q / H_kv,
+                                          reinterpret_cast<unsigned long long*>(ws + kWsLivePairs),
+                                          reinterpret_cast<int*>(ws + kWsHeader));
+  return cudaGetLastError() == cudaSuccess ? EA_OK : EA_ERR_CUDA;
+}
+
+}  // namespace ea
