@@ -1,0 +1,451 @@
+"""Benchmark of the Elastic Attention prefill path (one layer) on B200.
+
+One step = the whole hot path on one batch of synthetic inputs already in HBM:
+router (boundary pooling + head MLP + threshold) -> device work list -> hybrid
+attention launch -> sparsity report.  Default workload: the Llama-3.1-8B-shaped
+layer at S = 32768 (B=1, D=4096, H_q=32, H_kv=8, d=128, bf16, streaming sparse
+heads with 128 sinks and a 2048 window, router tuned to Omega_MSR = 50%).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Prints one JSON line (rank 0).  value = live-tile TFLOP/s of the whole step
+(4*d*128^2 per live 128x128 tile per query head, divided by the step time).
+Multi-GPU: one process per GPU, each runs its own replica of the layer (the
+work partitions by (sample, KV head) with no exchange), scaling "weak".
+--impl reference times the CPU oracle on a bounded sample of the same
+workload (the reference arm: a deliberately slow program).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "llama3-8b-s32k-streaming"
+
+# DRAM bytes (read + write) of one attention launch from an ncu capture, keyed by the
+# hash of the kernel's sources: a changed kernel reports traffic null until re-measured.
+ATTN_SOURCES = ("sparse_gqa_attention_b200/csrc/ea_attn_tc.cu", "sparse_gqa_attention_b200/csrc/ea_common.cuh",
+                "sparse_gqa_attention_b200/csrc/ea_sm100.cuh")
+ATTN_TRAFFIC = {  # source hash -> {workload: bytes per launch}
+    "61541492d61925e1": {"llama3-8b-s32k-streaming": 594458112 + 241475584},
+}
+
+
+def attn_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ATTN_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+METRIC = "hybrid prefill TFLOP/s on live tiles & tokens/s at S=32k–128k, % of BF16 peak"
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            m = json.load(f)
+        return dict(hbm=float(m["hbm_gbs"]), bf16=float(m["bf16_tflops"]),
+                    bf16_sustained=float(m["bf16_tflops_sustained"]), source="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            self.proc.wait(timeout=5)
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[3:7]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def make_inputs(w):
+    import workloads as wl
+    q, k, v = wl.attention_inputs(w)
+    return dict(hidden=wl.hidden_states(w), weights=wl.router_weights(w), q=q, k=k, v=v,
+                pattern=wl.pattern_for(w))
+
+
+def to_torch(x, dtype_name):
+    import torch
+    if dtype_name == "bf16" and x.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(x))
+
+
+# ---------------------------------------------------------------------------- CUDA arm
+
+def run_cuda(args):
+    import torch
+    import torch.distributed as dist
+
+    import workloads as wl
+    from sparse_gqa_attention_b200 import abi
+    import __graft_entry__
+
+    world, rank, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    __graft_entry__.build()
+    w = wl.WORKLOADS[args.workload]
+    inp = make_inputs(w)
+    dev = torch.device("cuda", local)
+    st = torch.cuda.current_stream()
+
+    hidden = to_torch(inp["hidden"], w.dtype).to(dev)
+    weights = {k: to_torch(v, w.dtype).to(dev) for k, v in inp["weights"].items()}
+    q, k, v = (to_torch(x, w.dtype).to(dev) for x in (inp["q"], inp["k"], inp["v"]))
+    o = torch.empty_like(q)
+    pat = abi.Pattern.from_workloads(inp["pattern"])
+    head_mode = torch.zeros(w.B, w.H_kv, dtype=torch.int32, device=dev)
+    rws = torch.zeros(abi.ea_router_workspace_size(w.B, w.S, w.D, w.n_boundary), dtype=torch.uint8, device=dev)
+    aws = torch.zeros(abi.ea_attn_workspace_size(w.B, w.S, w.H_q, w.H_kv), dtype=torch.uint8, device=dev)
+    forced = None
+    if args.omega_sparse is not None:
+        forced = torch.from_numpy(wl.forced_head_mode(w, args.omega_sparse)).to(dev)
+
+    ev = {n: [] for n in ("r0", "r1", "a0", "a1", "a2")}
+    report = {}
+
+    def step(record):
+        if record:
+            e = torch.cuda.Event(enable_timing=True); e.record(st); ev["r0"].append(e)
+        abi.ea_router(hidden, weights, head_mode, rws, w.n_boundary)
+        hm = head_mode if forced is None else forced
+        if record:
+            e = torch.cuda.Event(enable_timing=True); e.record(st); ev["r1"].append(e)
+        abi.ea_build_schedule(hm, pat, w.B, w.S, w.H_q, w.H_kv, w.d, aws)
+        if record:
+            e = torch.cuda.Event(enable_timing=True); e.record(st); ev["a1"].append(e)
+        abi.ea_attn_scheduled(q, k, v, hm, pat, o, aws)
+        if record:
+            e = torch.cuda.Event(enable_timing=True); e.record(st); ev["a2"].append(e)
+        per, rep = abi.ea_effective_sparsity(hm, pat, w.B, w.S, w.H_q, w.H_kv, w.d, aws)
+        report["per"], report["rep"] = per, rep
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        t0.record(st)
+        for _ in range(args.steps):
+            step(True)
+        t1.record(st)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    ms_total = t0.elapsed_time(t1)
+    status = abi.ea_workspace_status(aws)
+    if status != abi.EA_OK:
+        raise RuntimeError(f"device status after the timed steps: {abi.ea_status_string(status)}")
+    attn_ms = [a.elapsed_time(b) for a, b in zip(ev["a1"], ev["a2"])]
+    router_ms = [a.elapsed_time(b) for a, b in zip(ev["r0"], ev["r1"])]
+    sched_ms = [a.elapsed_time(b) for a, b in zip(ev["r1"], ev["a1"])]
+    rep = report["rep"]
+    live_flops = rep["live_flops"]
+
+    # End to end through the same ABI: pinned host inputs -> device, step, result -> host.
+    e2e = e2e_measure(args, w, inp, dev, st, weights, pat, forced, rws, aws)
+
+    # Router pooling over the whole sequence (bandwidth measurement).
+    router_full = router_bandwidth(w, hidden, weights, dev, st)
+
+    t_max = ms_total
+    if world > 1:
+        tt = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max = float(tt.item())
+        et = torch.tensor([e2e["ms_per_step"]], device=dev, dtype=torch.float64)
+        dist.all_reduce(et, op=dist.ReduceOp.MAX)
+        e2e["ms_per_step"] = float(et.item())
+    ms_step = t_max / args.steps
+    pk = peaks()
+    attn_avg = statistics.mean(attn_ms)
+    achieved = live_flops / (attn_avg * 1e-3) / 1e12
+    value = world * live_flops / (ms_step * 1e-3) / 1e12
+    tokens = w.B * w.S
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,1); no dataset, random router)",
+            "config": {"workload": w.name, "B": w.B, "S": w.S, "D": w.D, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d,
+                       "n_sink": w.n_sink, "window": w.window,
+                       "omega_msr": float(np.mean(report["per"])), "omega_esr": round(rep["omega_esr"], 6),
+                       "forced_sparse_kv_heads": args.omega_sparse,
+                       "l2": "inputs larger than L2 (q+k+v+hidden > 126 MB), no explicit flush",
+                       "parallelism": f"replica x{world}"},
+            "tokens_per_s": round(world * tokens / (ms_step * 1e-3), 1),
+            "tflops_dense_causal_equiv": round(world * 4 * w.d * w.H_q * w.B * w.S * (w.S + 1) / 2
+                                               / (ms_step * 1e-3) / 1e12, 2),
+            "kernels_ms": {"router": round(statistics.mean(router_ms), 4),
+                           "schedule": round(statistics.mean(sched_ms), 4),
+                           "attention": round(attn_avg, 4)},
+            "roofline": {"bound": "tensor", "kernel": "hybrid_attn_tc_kernel", "achieved": round(achieved, 2),
+                         "peak": pk["bf16"], "unit": "TFLOP/s", "frac": round(achieved / pk["bf16"], 4),
+                         "peak_source": f"bf16_tflops burst, {pk['source']}",
+                         "frac_of_sustained": round(achieved / pk["bf16_sustained"], 4),
+                         "traffic": ATTN_TRAFFIC.get(attn_source_hash(), {}).get(w.name),
+                         "algorithmic_bytes": int(2 * w.B * w.S * w.d * (2 * w.H_q + 2 * w.H_kv))},
+            "router_roofline": router_full,
+            "e2e": e2e,
+            "gpu_launches": 6 * args.steps,
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, inp, live_flops, budget_s=args.cpu_budget)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def e2e_measure(args, w, inp, dev, st, weights, pat, forced, rws, aws):
+    import torch
+    from sparse_gqa_attention_b200 import abi
+    host = {n: to_torch(inp[n], w.dtype).pin_memory() for n in ("hidden", "q", "k", "v")}
+    dbuf = {n: torch.empty_like(t, device=dev) for n, t in host.items()}
+    o_dev = torch.empty_like(dbuf["q"])
+    o_host = torch.empty_like(host["q"]).pin_memory()
+    head_mode = torch.zeros(w.B, w.H_kv, dtype=torch.int32, device=dev)
+
+    def step():
+        for n in host:
+            dbuf[n].copy_(host[n], non_blocking=True)
+        abi.ea_router(dbuf["hidden"], weights, head_mode, rws, w.n_boundary)
+        hm = head_mode if forced is None else forced
+        abi.ea_hybrid_attn_prefill(dbuf["q"], dbuf["k"], dbuf["v"], hm, pat, o_dev, aws)
+        o_host.copy_(o_dev, non_blocking=True)
+        per, rep = abi.ea_effective_sparsity(hm, pat, w.B, w.S, w.H_q, w.H_kv, w.d, aws)  # synchronises
+        return rep
+
+    for _ in range(max(1, min(args.warmup, 3))):
+        rep = step()
+    torch.cuda.synchronize()
+    n = max(2, min(args.steps, 5))
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(st)
+    for _ in range(n):
+        rep = step()
+    t1.record(st)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / n
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    return {"value": round(rep["live_flops"] / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s", "ms_per_step": ms,
+            "steps": n, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(o_host.numel() * o_host.element_size() + 4 * w.B + 32),
+            "api": "ea_router + ea_hybrid_attn_prefill + ea_effective_sparsity on pinned host buffers"}
+
+
+def router_bandwidth(w, hidden, weights, dev, st):
+    import torch
+    from sparse_gqa_attention_b200 import abi
+    ws = torch.zeros(abi.ea_router_workspace_size(w.B, w.S, w.D, 0), dtype=torch.uint8, device=dev)
+    hm = torch.zeros(w.B, w.H_kv, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    times = []
+    for it in range(8):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        abi.ea_router(hidden, weights, hm, ws, 0)
+        b.record(st)
+        torch.cuda.synchronize()
+        if it >= 3:
+            times.append(a.elapsed_time(b))
+    bytes_ = hidden.numel() * hidden.element_size() + weights["w_k"].numel() * weights["w_k"].element_size()
+    ms = statistics.median(times)
+    gbs = bytes_ / (ms * 1e-3) / 1e9
+    pk = peaks()
+    boundary = []
+    ws_b = torch.zeros(abi.ea_router_workspace_size(w.B, w.S, w.D, w.n_boundary), dtype=torch.uint8, device=dev)
+    for it in range(8):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        abi.ea_router(hidden, weights, hm, ws_b, w.n_boundary)
+        b.record(st)
+        torch.cuda.synchronize()
+        if it >= 3:
+            boundary.append(a.elapsed_time(b))
+    del flush
+    return {"bound": "hbm", "mode": "full-sequence pooling (n_boundary=0)", "achieved": round(gbs, 1),
+            "peak": pk["hbm"], "unit": "GB/s", "frac": round(gbs / pk["hbm"], 4), "bytes": int(bytes_),
+            "ms": round(ms, 4), "boundary_mode_us": round(1e3 * statistics.median(boundary), 2)}
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample(w, inp, budget_s):
+    """Time the oracle on a bounded sample: the router in full (boundary pooling)
+    plus attention rows of every query head until ~budget_s of CPU time; the
+    rows are spread evenly over the sequence so the per-row cost is
+    representative.  Returns (seconds for the full workload, extrapolated, and
+    the sample description)."""
+    import oracle
+    import workloads as wl
+    f64 = lambda x: (wl.f32_from_bf16_bits(x) if x.dtype == np.uint16 else x).astype(np.float64)  # noqa: E731
+    t0 = time.perf_counter()
+    hw = dict(inp["weights"])
+    hw["w_k"] = f64(hw["w_k"])
+    h32 = wl.f32_from_bf16_bits(inp["hidden"]) if inp["hidden"].dtype == np.uint16 else inp["hidden"]
+    _, mode = oracle.router.router_forward(h32, hw, w.H_kv, w.d, w.n_boundary)
+    t_router = time.perf_counter() - t0
+    pat = inp["pattern"]
+    pd = dict(n_sink=pat.n_sink, window=pat.window, block=pat.block, row_ptr=pat.row_ptr, cols=pat.cols,
+              kind_if_dense=pat.kind_if_dense, kind_if_sparse=pat.kind_if_sparse)
+    k64, v64 = f64(inp["k"]), f64(inp["v"])
+    rows_done, t_attn, n_rows = 0, 0.0, 4
+    while t_attn < budget_s and rows_done < w.S:
+        rows = np.unique(np.linspace(0, w.S - 1, n_rows).astype(np.int64) + rows_done % 7)
+        rows = rows[rows < w.S]
+        t1 = time.perf_counter()
+        oracle.attention.hybrid_attention_rows(f64(inp["q"][:, rows]), k64, v64, mode, pd, rows, q_row_index=rows)
+        t_attn += time.perf_counter() - t1
+        rows_done += len(rows)
+        n_rows *= 2
+    per_row = t_attn / rows_done           # all B x H_q heads of one row position
+    total = t_router + per_row * w.S
+    sample = (f"router in full + attention on {rows_done} row positions (all {w.B}x{w.H_q} heads, spread over "
+              f"S={w.S}); full-workload time extrapolated as router + per-row time x S")
+    return total, sample
+
+
+def cpu_baseline(w, inp, live_flops, budget_s=15.0):
+    total, sample = oracle_sample(w, inp, budget_s)
+    return {"value": round(live_flops / total / 1e12, 8), "unit": "TFLOP/s", "cores": cpu_threads(),
+            "kind": "oracle", "sample": sample, "seconds_extrapolated": round(total, 2)}
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return
+    import workloads as wl
+    import oracle
+    w = wl.WORKLOADS[args.workload]
+    inp = make_inputs(w)
+    mode = wl.routing_targets(w)[2]
+    pat = inp["pattern"]
+    pd = dict(n_sink=pat.n_sink, window=pat.window, block=pat.block, row_ptr=pat.row_ptr, cols=pat.cols,
+              kind_if_dense=pat.kind_if_dense, kind_if_sparse=pat.kind_if_sparse)
+    live_flops = oracle.sparsity.sparsity_report(mode, pd, w.B, w.S, w.H_q, w.H_kv, w.d)["live_flops"]
+    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    times, sample = [], ""
+    for i in range(args.warmup + args.steps):
+        total, sample = oracle_sample(w, inp, budget)
+        if i >= args.warmup:
+            times.append(total)
+    sec = statistics.mean(times)
+    value = live_flops / sec / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 8), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1))",
+            "config": {"workload": w.name, "B": w.B, "S": w.S, "D": w.D, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d},
+            "cpu_baseline": {"value": round(value, 8), "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 8), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--omega-sparse", type=int, default=None, help="force this many sparse KV heads per sample")
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_cuda(args)
+
+
+if __name__ == "__main__":
+    main()

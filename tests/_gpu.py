@@ -1,6 +1,8 @@
 """Helpers for the GPU parity tests: device copies of the seeded inputs, calls
 through the C ABI, and the oracle on the same inputs (sampled rows for the
 full-size workloads)."""
+import functools
+
 import numpy as np
 import torch
 
@@ -9,6 +11,14 @@ import workloads as wl
 from sparse_gqa_attention_b200 import abi
 
 BF16_MAX_ABS, BF16_MEAN_ABS, F32_MAX_ABS = 2e-2, 2e-3, 1e-4
+
+
+@functools.lru_cache(maxsize=1)
+def cached_inputs(name: str):
+    """(q, k, v, hidden, router weights) of a named workload, drawn once per process."""
+    w = wl.WORKLOADS[name]
+    q, k, v = wl.attention_inputs(w)
+    return q, k, v, wl.hidden_states(w), wl.router_weights(w)
 
 
 def to_dev(x: np.ndarray, dtype: str):

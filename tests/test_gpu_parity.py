@@ -37,7 +37,7 @@ def _built():
 @pytest.mark.parametrize("name", SMALL + FULL)
 def test_router_decisions_bit_exact(name):
     w = wl.WORKLOADS[name]
-    weights, hidden = wl.router_weights(w), wl.hidden_states(w)
+    _, _, _, hidden, weights = _gpu.cached_inputs(name)
     hm, z = _gpu.run_router(w, hidden, weights)
     z_ref, m_ref = _gpu.oracle_router(w, hidden, weights)
     np.testing.assert_array_equal(hm, m_ref)
@@ -123,7 +123,7 @@ def test_split_calls_equal_one_call_and_are_deterministic():
 @pytest.mark.parametrize("name", FULL)
 def test_full_size_sampled_rows(name):
     w = wl.WORKLOADS[name]
-    q, k, v = wl.attention_inputs(w)
+    q, k, v, _, _ = _gpu.cached_inputs(name)
     mode, pat = wl.routing_targets(w)[2], wl.pattern_for(w)
     rows = _gpu.sample_rows(w)
     got, status = _gpu.run_attention(w, q, k, v, mode, pat, rows=rows)
@@ -135,7 +135,7 @@ def test_full_size_sampled_rows(name):
 @pytest.mark.parametrize("n_sparse", [0, 2, 4, 6, 8])
 def test_omega_sweep_sampled_rows(n_sparse):
     w = wl.WORKLOADS["llama3-8b-s128k-sweep"]
-    q, k, v = wl.attention_inputs(w)
+    q, k, v, _, _ = _gpu.cached_inputs(w.name)
     pat = wl.pattern_for(w)
     mode = wl.forced_head_mode(w, n_sparse)
     rows = _gpu.sample_rows(w, n_random=6)
