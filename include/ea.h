@@ -109,6 +109,25 @@ EA_API ea_status ea_router(const void* hidden, ea_dtype dtype, int B, int S, int
                     int32_t* head_mode, float* logits,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* Router with library-owned scratch.  The paper has no counterpart: this is an
+ * interface for callers that cannot allocate device memory — a runtime or plugin
+ * host that owns every device allocation, or code running while a stream is
+ * captured (cudaMalloc is rejected during a global-mode capture and may
+ * synchronise the device).  Same arguments and outputs as ea_router, without
+ * the workspace: the scratch is a fixed EA_ROUTER_STATIC_SCRATCH_BYTES array
+ * inside the library, held on every GPU that loads it until the process exits.
+ * It allocates nothing (no cudaMalloc, cudaFree or allocating library call).
+ * Problems whose scratch (ea_router_workspace_size) exceeds the array return
+ * EA_ERR_INVALID_ARG before any launch.  The first call on each device looks
+ * up the array's device address; make that first call before any stream
+ * capture.  All calls share the array: calls that overlap on the GPU race, so
+ * order them on one stream.  Nothing in the array needs to start at zero. */
+#define EA_ROUTER_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
+EA_API ea_status ea_router_static_scratch(const void* hidden, ea_dtype dtype, int B, int S, int D, int H_kv,
+                                          int d, const ea_router_weights* weights,
+                                          const ea_router_params* params, int32_t* head_mode, float* logits,
+                                          void* stream);
+
 /* ------------------------------------------------------------------------
  * Hybrid-head attention (section 2 "Hybrid Head Mechanism"; section 3
  * "Efficient Deployment"; appendix D.1 "Sparse Inference": the routing

@@ -85,6 +85,10 @@ def _lib():
         lib.ea_effective_sparsity.restype = st
         lib.ea_effective_sparsity.argtypes = [c_void_p, POINTER(PatternParams), c_int, c_int, c_int, c_int, c_int,
                                               c_void_p, POINTER(SparsityReport), c_void_p, c_size_t, c_void_p]
+        lib.ea_router_static_scratch.restype = st
+        lib.ea_router_static_scratch.argtypes = [c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
+                                                 POINTER(RouterWeights), POINTER(RouterParams), c_void_p,
+                                                 c_void_p, c_void_p]
         lib.ea_workspace_status.restype = st
         lib.ea_workspace_status.argtypes = [c_void_p, c_void_p]
         _LIB = lib
@@ -175,6 +179,24 @@ def ea_router(hidden: torch.Tensor, weights: dict, head_mode: torch.Tensor, work
                               _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
                               _stream(stream))
     _check(status, "ea_router")
+
+
+def ea_router_static_scratch(hidden: torch.Tensor, weights: dict, head_mode: torch.Tensor, n_boundary: int = 100,
+                             logits: torch.Tensor | None = None, stream=None):
+    """ea_router without a workspace: the library's fixed scratch array is used instead
+    (for callers that cannot allocate device memory; see include/ea.h)."""
+    B, S, D = hidden.shape
+    H_kv = weights["w_o"].shape[0]
+    d = weights["w_t1"].shape[1]
+    w = RouterWeights(*[_dev(weights[n], n) for n in
+                        ("w_k", "w_t1", "b_t1", "w_t2", "b_t2", "w_r1", "b_r1", "w_o", "b_o")])
+    prm = RouterParams(n_boundary)
+    status = _lib().ea_router_static_scratch(_dev(hidden, "hidden"), _dtype_code(hidden), B, S, D, H_kv, d,
+                                             ctypes.byref(w), ctypes.byref(prm),
+                                             _dev(head_mode, "head_mode", torch.int32),
+                                             _dev(logits, "logits", torch.float32) if logits is not None else None,
+                                             _stream(stream))
+    _check(status, "ea_router_static_scratch")
 
 
 # ---------------------------------------------------------------------------
