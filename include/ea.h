@@ -96,8 +96,8 @@ typedef struct {          /* all device pointers, row-major                   */
   const float* b_o;       /* [H_kv]    */
 } ea_router_weights;
 
-/* Bytes of workspace ea_router needs (pooling partial sums and hbar). */
-EA_API size_t ea_router_workspace_size(int B, int S, int D, int n_boundary);
+/* Bytes of workspace ea_router needs (pooling and key-projection partial sums). */
+EA_API size_t ea_router_workspace_size(int B, int S, int D, int H_kv, int d, int n_boundary);
 
 /* Router for one layer.  hidden: device [B, S, D] in `dtype`
  * (D % 8 == 0 for bf16, D % 4 == 0 for f32); d in {64, 128};

@@ -66,7 +66,7 @@ def _lib():
         lib.ea_status_string.restype = ctypes.c_char_p
         lib.ea_status_string.argtypes = [c_int]
         lib.ea_router_workspace_size.restype = c_size_t
-        lib.ea_router_workspace_size.argtypes = [c_int, c_int, c_int, c_int]
+        lib.ea_router_workspace_size.argtypes = [c_int, c_int, c_int, c_int, c_int, c_int]
         lib.ea_attn_workspace_size.restype = c_size_t
         lib.ea_attn_workspace_size.argtypes = [c_int, c_int, c_int, c_int]
         lib.ea_router.restype = st
@@ -160,8 +160,8 @@ class Pattern:
 # Router
 # ---------------------------------------------------------------------------
 
-def ea_router_workspace_size(B: int, S: int, D: int, n_boundary: int = 100) -> int:
-    return int(_lib().ea_router_workspace_size(B, S, D, n_boundary))
+def ea_router_workspace_size(B: int, S: int, D: int, H_kv: int, d: int, n_boundary: int = 100) -> int:
+    return int(_lib().ea_router_workspace_size(B, S, D, H_kv, d, n_boundary))
 
 
 def ea_router(hidden: torch.Tensor, weights: dict, head_mode: torch.Tensor, workspace: torch.Tensor,

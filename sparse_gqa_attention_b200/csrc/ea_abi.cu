@@ -75,9 +75,9 @@ ea_status check_ws(const void* ws, size_t bytes, size_t need) {
 
 extern "C" {
 
-size_t ea_router_workspace_size(int B, int S, int D, int n_boundary) {
-  if (B < 1 || S < 1 || D < 1) return 0;
-  return router_workspace_bytes(B, S, D, n_boundary);
+size_t ea_router_workspace_size(int B, int S, int D, int H_kv, int d, int n_boundary) {
+  if (B < 1 || S < 1 || D < 1 || H_kv < 1 || d < 1) return 0;
+  return router_workspace_bytes(B, S, D, H_kv, d, n_boundary);
 }
 
 ea_status ea_router(const void* hidden, ea_dtype dtype, int B, int S, int D, int H_kv, int d,
@@ -92,7 +92,7 @@ ea_status ea_router(const void* hidden, ea_dtype dtype, int B, int S, int D, int
   if (dtype != EA_DT_BF16 && dtype != EA_DT_F32) return EA_ERR_INVALID_ARG;
   if (D % (dtype == EA_DT_BF16 ? 8 : 4) != 0 || !aligned16(hidden)) return EA_ERR_INVALID_ARG;
   if ((size_t)D * sizeof(float) + 12u * d * sizeof(float) > 200u * 1024u) return EA_ERR_UNSUPPORTED;
-  if (ea_status s = check_ws(workspace, workspace_bytes, router_workspace_bytes(B, S, D, prm->n_boundary)))
+  if (ea_status s = check_ws(workspace, workspace_bytes, router_workspace_bytes(B, S, D, H_kv, d, prm->n_boundary)))
     return s;
   return launch_router(hidden, dtype, B, S, D, H_kv, d, w, prm, head_mode, logits, workspace, as_stream(stream));
 }

@@ -12,9 +12,11 @@
 // a snake order.  A work item is 128 query rows of two query heads of one KV
 // group (two "slots"), so every K/V tile brought into shared memory feeds two
 // 128x128 products.  Warp roles, 384 threads:
-//   warp 0      TMA producer: Q tiles of both slots, then K and V tiles of each
-//               live key tile into an NST-stage ring (128-byte swizzle, 2 boxes
-//               of 64 columns per 128x128 tile).  No cluster multicast.
+//   warp 0      TMA producer: Q tiles of both slots, then the K and V tiles of each
+//               live key tile into separate rings (3 K stages, released as soon as
+//               both Q K^T products finish; 2 V stages, released after the P V
+//               products), 128-byte swizzle, 2 boxes of 64 columns per 128x128
+//               tile.  No cluster multicast.
 //   warp 1      TMEM owner and MMA issuer (one thread): S_s = Q_s K^T (SS MMA,
 //               M=N=128, K=16 steps) into TMEM, then O_s += P_s V (TS MMA: P
 //               read from TMEM, V from shared memory as an MN-major operand).
@@ -48,22 +50,23 @@ namespace {
 using namespace sm100;
 
 constexpr int BM = 128, BN = 128, HD = 128;
-constexpr int NST = 2;                                 // K/V stages
+constexpr int NK = 3, NV = 2;                          // K stages, V stages
 constexpr int kThreads = 384;
 constexpr uint32_t kTileBytes = BM * HD * 2;           // 32 KB per 128x128 bf16 tile
 constexpr uint32_t kBoxBytes = kTileBytes / 2;         // one 64-column box
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = 2 * kTileBytes;
-constexpr uint32_t OFF_V = OFF_K + NST * kTileBytes;
-constexpr uint32_t OFF_BAR = OFF_V + NST * kTileBytes;
+constexpr uint32_t OFF_V = OFF_K + NK * kTileBytes;
+constexpr uint32_t OFF_BAR = OFF_V + NV * kTileBytes;
 enum : int {
-  B_QFULL = 0, B_QEMPTY = 2, B_KFULL = 4, B_VFULL = B_KFULL + NST, B_KVEMPTY = B_VFULL + NST,
-  B_SFULL = B_KVEMPTY + NST, B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2, B_OFULL = B_PVDONE + 2,
-  B_FIN = B_OFULL + 2, N_BAR = B_FIN + 1
+  B_QFULL = 0, B_QEMPTY = 2, B_KFULL = 4, B_KEMPTY = B_KFULL + NK, B_VFULL = B_KEMPTY + NK,
+  B_VEMPTY = B_VFULL + NV, B_SFULL = B_VEMPTY + NV, B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2,
+  B_OFULL = B_PVDONE + 2, B_FIN = B_OFULL + 2, N_BAR = B_FIN + 1
 };
 constexpr uint32_t OFF_TMEM = OFF_BAR + N_BAR * 8;
 constexpr uint32_t OFF_ABORT = OFF_TMEM + 4;
 constexpr uint32_t kSmemBytes = OFF_ABORT + 4 + 1024;  // + slack to align the base to 1024
+static_assert(kSmemBytes <= 232448, "shared memory beyond the 227 KB a CTA may use");
 constexpr uint32_t kTmemCols = 512;
 __device__ __forceinline__ uint32_t col_s(int s) { return 128u * s; }        // S_s (and P_s) columns
 __device__ __forceinline__ uint32_t col_o(int s) { return 256u + 128u * s; } // O_s columns
@@ -71,6 +74,7 @@ constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, false);
 constexpr uint32_t IDESC_PV = idesc_bf16(BM, HD, true);
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr float kRescaleLog2 = 8.0f;
+
 // Register split: the launch gives 384 x 168 = 64512 registers; warpgroup 0 (producer,
 // MMA, two idle warps) drops to 88 and the two softmax warpgroups rise to 208:
 // 128 x 88 + 256 x 208 = 64512.
@@ -194,9 +198,17 @@ __device__ __forceinline__ float softmax_tile(const float (&x)[BN], int lim, int
     if (kMode == 1) return e <= lim;
     return e <= lim && (e < sink_lim || e > win_lim);
   };
-  float mt = -INFINITY;
+  auto xm = [&](int e) { return live(e) ? x[e] : -INFINITY; };
+  // Row max as 8 independent 3-input chains over 16 columns each, then a short tree.
+  float m8[8];
 #pragma unroll
-  for (int e = 0; e < BN; ++e) mt = fmaxf(mt, live(e) ? x[e] : -INFINITY);
+  for (int c = 0; c < 8; ++c) {
+    m8[c] = xm(16 * c);
+#pragma unroll
+    for (int e = 1; e + 1 < 16; e += 2) m8[c] = fmax3(m8[c], xm(16 * c + e), xm(16 * c + e + 1));
+    m8[c] = fmaxf(m8[c], xm(16 * c + 15));
+  }
+  const float mt = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
   const float mts = mt * scale_log2;
   float f = 1.f;
   if (mts > m_ref + kRescaleLog2) {
@@ -205,19 +217,26 @@ __device__ __forceinline__ float softmax_tile(const float (&x)[BN], int lim, int
     m_ref = mts;
   }
   const float sub = (m_ref == -INFINITY) ? 0.f : m_ref;
+  const uint64_t scale2 = f2_pack(scale_log2, scale_log2), nsub2 = f2_pack(-sub, -sub);
+  uint64_t l2 = f2_pack(0.f, 0.f);
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     uint32_t pk[32];
 #pragma unroll
     for (int e = 0; e < 64; e += 2) {
       const int e0 = 64 * half + e;
-      const float p0 = live(e0) ? ex2(fmaf(x[e0], scale_log2, -sub)) : 0.f;
-      const float p1 = live(e0 + 1) ? ex2(fmaf(x[e0 + 1], scale_log2, -sub)) : 0.f;
-      l += p0 + p1;
+      float t0, t1;
+      f2_unpack(f2_fma(f2_pack(x[e0], x[e0 + 1]), scale2, nsub2), t0, t1);
+      const float p0 = live(e0) ? ex2(t0) : 0.f;
+      const float p1 = live(e0 + 1) ? ex2(t1) : 0.f;
+      l2 = f2_add(l2, f2_pack(p0, p1));
       pk[e / 2] = pack_bf16x2(p0, p1);
     }
     tmem_st32(p_addr + 32 * half, pk);
   }
+  float la, lb;
+  f2_unpack(l2, la, lb);
+  l += la + lb;
   return f;
 }
 
@@ -263,7 +282,7 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int q_use[2] = {0, 0};
-      int kv_it = 0;
+      int k_it = 0, v_it = 0;
       bool ok = true;
       for (int it = 0; ok; ++it) {
         const int idx = item_index(it, blockIdx.x, gridDim.x);
@@ -284,26 +303,31 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         for (int jj = 0; jj < I.n && ok; ++jj) {
           const int ct = max(0, live_tile(p, I.kind, I.t, jj, I.sink_end, I.win_lo, I.csr_beg));
-          const int st = kv_it % NST;
-          ok = wait(c, c.bar(B_KVEMPTY + st), ((kv_it / NST) & 1) ^ 1);
+          const int ks = k_it % NK, vs = v_it % NV;
+          ok = wait(c, c.bar(B_KEMPTY + ks), ((k_it / NK) & 1) ^ 1);
           if (!ok) break;
-          const uint32_t kdst = base + OFF_K + st * kTileBytes, vdst = base + OFF_V + st * kTileBytes;
-          mbar_expect_tx(c.bar(B_KFULL + st), kTileBytes);
-          tma_load_4d(kdst, &tm_k, c.bar(B_KFULL + st), 0, I.h, ct * BN, I.b);
-          tma_load_4d(kdst + kBoxBytes, &tm_k, c.bar(B_KFULL + st), 64, I.h, ct * BN, I.b);
-          mbar_expect_tx(c.bar(B_VFULL + st), kTileBytes);
-          tma_load_4d(vdst, &tm_v, c.bar(B_VFULL + st), 0, I.h, ct * BN, I.b);
-          tma_load_4d(vdst + kBoxBytes, &tm_v, c.bar(B_VFULL + st), 64, I.h, ct * BN, I.b);
-          ++kv_it;
+          const uint32_t kdst = base + OFF_K + ks * kTileBytes;
+          mbar_expect_tx(c.bar(B_KFULL + ks), kTileBytes);
+          tma_load_4d(kdst, &tm_k, c.bar(B_KFULL + ks), 0, I.h, ct * BN, I.b);
+          tma_load_4d(kdst + kBoxBytes, &tm_k, c.bar(B_KFULL + ks), 64, I.h, ct * BN, I.b);
+          ++k_it;
+          ok = wait(c, c.bar(B_VEMPTY + vs), ((v_it / NV) & 1) ^ 1);
+          if (!ok) break;
+          const uint32_t vdst = base + OFF_V + vs * kTileBytes;
+          mbar_expect_tx(c.bar(B_VFULL + vs), kTileBytes);
+          tma_load_4d(vdst, &tm_v, c.bar(B_VFULL + vs), 0, I.h, ct * BN, I.b);
+          tma_load_4d(vdst + kBoxBytes, &tm_v, c.bar(B_VFULL + vs), 64, I.h, ct * BN, I.b);
+          ++v_it;
         }
       }
       // Drain: the last copy armed on every barrier has landed before the CTA exits.
-      for (int st = 0; st < NST; ++st) {
-        const int uses = kv_it / NST + (st < kv_it % NST ? 1 : 0);
-        if (uses > 0) {
-          wait_slow(c, c.bar(B_KFULL + st), (uses - 1) & 1);
-          wait_slow(c, c.bar(B_VFULL + st), (uses - 1) & 1);
-        }
+      for (int st = 0; st < NK; ++st) {
+        const int uses = k_it / NK + (st < k_it % NK ? 1 : 0);
+        if (uses > 0) wait_slow(c, c.bar(B_KFULL + st), (uses - 1) & 1);
+      }
+      for (int st = 0; st < NV; ++st) {
+        const int uses = v_it / NV + (st < v_it % NV ? 1 : 0);
+        if (uses > 0) wait_slow(c, c.bar(B_VFULL + st), (uses - 1) & 1);
       }
 #pragma unroll
       for (int s = 0; s < 2; ++s)
@@ -314,7 +338,7 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (lane == 0) {
       int q_use0 = 0, q_use1 = 0, p_cnt0 = 0, p_cnt1 = 0, pv_cnt0 = 0, pv_cnt1 = 0;
       bool pend0 = false, pend1 = false;
-      int kv_it = 0;
+      int k_it = 0, v_it = 0;
       bool ok = true;
       for (int it = 0; ok; ++it) {
         const int idx = item_index(it, blockIdx.x, gridDim.x);
@@ -327,26 +351,33 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           ok = ok && wait(c, c.bar(B_QFULL + 1), q_use1 & 1);
           ++q_use1;
         }
-        ok = ok && wait(c, c.bar(B_KFULL + kv_it % NST), (kv_it / NST) & 1);
+        // S of the item's first key tile; its K stage is released once both products finish.
+        ok = ok && wait(c, c.bar(B_KFULL + k_it % NK), (k_it / NK) & 1);
         if (ok) {
-          ok = issue_qk<kSafeAlias>(c, tmem, base, 0, kv_it % NST, pend0, pv_cnt0);
-          if (ok && I.two) ok = issue_qk<kSafeAlias>(c, tmem, base, 1, kv_it % NST, pend1, pv_cnt1);
+          ok = issue_qk<kSafeAlias>(c, tmem, base, 0, k_it % NK, pend0, pv_cnt0);
+          if (ok && I.two) ok = issue_qk<kSafeAlias>(c, tmem, base, 1, k_it % NK, pend1, pv_cnt1);
+          commit(c.bar(B_KEMPTY + k_it % NK));
+          ++k_it;
         }
         for (int jj = 0; jj < I.n && ok; ++jj) {
-          const int st = kv_it % NST, st1 = (kv_it + 1) % NST;
+          const int vs = v_it % NV, ks = k_it % NK;
           const bool last = jj + 1 == I.n;
-          ok = wait(c, c.bar(B_VFULL + st), (kv_it / NST) & 1);
-          if (ok) ok = issue_pv(c, tmem, base, 0, st, jj > 0, last, p_cnt0, pv_cnt0, pend0);
+          ok = wait(c, c.bar(B_VFULL + vs), (v_it / NV) & 1);
+          if (ok) ok = issue_pv(c, tmem, base, 0, vs, jj > 0, last, p_cnt0, pv_cnt0, pend0);
           if (ok && !last) {
-            ok = wait(c, c.bar(B_KFULL + st1), ((kv_it + 1) / NST) & 1);
-            if (ok) ok = issue_qk<kSafeAlias>(c, tmem, base, 0, st1, pend0, pv_cnt0);
+            ok = wait(c, c.bar(B_KFULL + ks), (k_it / NK) & 1);
+            if (ok) ok = issue_qk<kSafeAlias>(c, tmem, base, 0, ks, pend0, pv_cnt0);
           }
           if (ok && I.two) {
-            ok = issue_pv(c, tmem, base, 1, st, jj > 0, last, p_cnt1, pv_cnt1, pend1);
-            if (ok && !last) ok = issue_qk<kSafeAlias>(c, tmem, base, 1, st1, pend1, pv_cnt1);
+            ok = issue_pv(c, tmem, base, 1, vs, jj > 0, last, p_cnt1, pv_cnt1, pend1);
+            if (ok && !last) ok = issue_qk<kSafeAlias>(c, tmem, base, 1, ks, pend1, pv_cnt1);
           }
-          commit(c.bar(B_KVEMPTY + st));
-          ++kv_it;
+          if (!last) {
+            commit(c.bar(B_KEMPTY + ks));   // K tile jj+1: both Q K^T products issued
+            ++k_it;
+          }
+          commit(c.bar(B_VEMPTY + vs));     // V tile jj: both P V products issued
+          ++v_it;
         }
       }
       commit(c.bar(B_FIN));                       // every MMA issued here has completed
@@ -446,6 +477,7 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   fence_before_sync();
   __syncthreads();
   if (warp == 1) {
+    __syncwarp();
     fence_after_sync();
     tmem_dealloc(tmem, kTmemCols);
   }

@@ -8,7 +8,7 @@
 namespace ea {
 struct PatternDev;
 
-size_t router_workspace_bytes(int B, int S, int D, int n_boundary);
+size_t router_workspace_bytes(int B, int S, int D, int H_kv, int d, int n_boundary);
 ea_status launch_router(const void* hidden, ea_dtype dtype, int B, int S, int D, int H_kv, int d,
                         const ea_router_weights* w, const ea_router_params* prm, int32_t* head_mode,
                         float* logits, void* workspace, cudaStream_t st);

@@ -5,12 +5,13 @@
 // states -> task MLP -> router MLP -> head-wise logit, hard decision), appendix
 // H.4 "Router Input Length" (first and last 100 tokens), section 5 (x4 width).
 //
-// Kernels:
-//   pool_partial   HBM-bound streaming reduction of hidden rows: 16-byte vector
-//                  loads, fp32 accumulation, one partial sum per (split, b, column).
-//   pool_finish    sums the partials in a fixed order and divides by |pooled rows|.
-//   router_mlp     one CTA per (KV head, sample): key projection GEMV over D, task
-//                  MLP, router MLP, output row, threshold.  Warp-per-row dot products.
+// Kernels (all fp32 arithmetic, fixed summation orders, so results are reproducible):
+//   pool_partial   HBM-bound streaming reduction of the pooled hidden rows: 16-byte
+//                  loads, 8 in flight per thread, one partial sum per (split, b, column).
+//   project        one CTA per 64 rows of W_k: finishes the pooled mean of its rows,
+//                  then the partial key projections of those rows for every column.
+//   router_mlp     one CTA per (KV head, sample): sums the projection partials of its
+//                  head, task MLP, router MLP on [p; tau], output row, threshold.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
@@ -54,7 +55,7 @@ __device__ __forceinline__ int pooled_token(int n, int a_len, int b_start) {
 }
 
 // grid (column chunks, splits, B); each thread sums VEC consecutive columns over the
-// split's rows with 4 independent 16-byte loads in flight.
+// split's rows with 8 independent 16-byte loads in flight.
 template <typename T>
 __global__ void __launch_bounds__(kPoolThreads)
 pool_partial_kernel(const T* __restrict__ hidden, int S, int D, int n_rows, int a_len, int b_start,
@@ -70,12 +71,12 @@ pool_partial_kernel(const T* __restrict__ hidden, int S, int D, int n_rows, int 
   if (col < D) {
     const T* base = hidden + (size_t)b * S * D + col;
     int n = r0;
-    for (; n + 4 <= r1; n += 4) {
-      uint4 x0 = ld_stream(base + (size_t)pooled_token(n, a_len, b_start) * D);
-      uint4 x1 = ld_stream(base + (size_t)pooled_token(n + 1, a_len, b_start) * D);
-      uint4 x2 = ld_stream(base + (size_t)pooled_token(n + 2, a_len, b_start) * D);
-      uint4 x3 = ld_stream(base + (size_t)pooled_token(n + 3, a_len, b_start) * D);
-      add_vec<T>(acc, x0); add_vec<T>(acc, x1); add_vec<T>(acc, x2); add_vec<T>(acc, x3);
+    for (; n + 8 <= r1; n += 8) {
+      uint4 x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = ld_stream(base + (size_t)pooled_token(n + u, a_len, b_start) * D);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) add_vec<T>(acc, x[u]);
     }
     for (; n < r1; ++n) add_vec<T>(acc, ld_stream(base + (size_t)pooled_token(n, a_len, b_start) * D));
     float* out = partial + ((size_t)split * gridDim.z + b) * D + col;
@@ -85,17 +86,123 @@ pool_partial_kernel(const T* __restrict__ hidden, int S, int D, int n_rows, int 
   }
 }
 
-__global__ void pool_finish_kernel(const float* __restrict__ partial, int n_splits, int B, int D,
-                                   float inv_rows, float* __restrict__ hbar) {
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= B * D) return;
-  float s = 0.f;
-  for (int sp = 0; sp < n_splits; ++sp) s += partial[(size_t)sp * B * D + idx];
-  hbar[idx] = s * inv_rows;
+constexpr int kProjRows = 64;      // rows of W_k per projection CTA
+constexpr int kProjThreads = 256;
+constexpr int kProjB = 4;          // samples per pass over a W_k chunk
+
+template <typename T>
+__device__ __forceinline__ void fma_vec(float* acc, uint4 raw, float x) {
+  if constexpr (Vec<T>::N == 4) {
+    acc[0] = fmaf(__uint_as_float(raw.x), x, acc[0]); acc[1] = fmaf(__uint_as_float(raw.y), x, acc[1]);
+    acc[2] = fmaf(__uint_as_float(raw.z), x, acc[2]); acc[3] = fmaf(__uint_as_float(raw.w), x, acc[3]);
+  } else {
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc[2 * e] = fmaf(__uint_as_float(w[e] << 16), x, acc[2 * e]);
+      acc[2 * e + 1] = fmaf(__uint_as_float(w[e] & 0xffff0000u), x, acc[2 * e + 1]);
+    }
+  }
 }
 
-constexpr int kMlpThreads = 256;
+// grid (ceil(D / kProjRows)).  For rows [r0, r0 + 64) of W_k:
+//   hbar[b][r] = (sum over splits of the pooling partial sums) / n_rows      (fixed order)
+//   pp[chunk][b][n] = sum_{r in chunk} W_k[r, n] * hbar[b][r]   for every column n < N = H_kv*d
+template <typename T>
+__global__ void __launch_bounds__(kProjThreads)
+project_kernel(const float* __restrict__ partial, int n_splits, int B, int D, float inv_rows,
+               const T* __restrict__ w_k, int N, float* __restrict__ pp) {
+  constexpr int V = Vec<T>::N;
+  __shared__ float hb[kProjB][kProjRows];
+  __shared__ float red[kProjThreads / kProjRows][kProjRows];
+  __shared__ float accs[kProjThreads * V];
+  const int r0 = blockIdx.x * kProjRows, tid = threadIdx.x;
+  const int rows = min(kProjRows, D - r0);
+  const int col_threads = N / V;                          // N % V == 0 (d in {64, 128})
+  for (int b0 = 0; b0 < B; b0 += kProjB) {
+    const int nb = min(kProjB, B - b0);
+    // Pooled hidden states of this chunk: thread = (row, split lane).
+    {
+      const int rl = tid % kProjRows, sl = tid / kProjRows, lanes = kProjThreads / kProjRows;
+      for (int bb = 0; bb < nb; ++bb) {
+        float s0 = 0.f, s1 = 0.f;
+        if (rl < rows) {
+          const float* src = partial + (size_t)(b0 + bb) * D + r0 + rl;
+          int sp = sl;
+          for (; sp + lanes < n_splits; sp += 2 * lanes) {
+            s0 += src[(size_t)sp * B * D];
+            s1 += src[(size_t)(sp + lanes) * B * D];
+          }
+          if (sp < n_splits) s0 += src[(size_t)sp * B * D];
+        }
+        red[sl][rl] = s0 + s1;
+        __syncthreads();
+        if (tid < kProjRows) {
+          float t = 0.f;
+          for (int l = 0; l < lanes; ++l) t += red[l][tid];
+          hb[bb][tid] = t * inv_rows;
+        }
+        __syncthreads();
+      }
+    }
+    // Partial projections: thread = (column group of V, row lane); columns loop when N/V > threads.
+    for (int c0 = 0; c0 < col_threads; c0 += kProjThreads) {
+      const int cgroups = min(kProjThreads, col_threads - c0);
+      const int lanes = max(1, kProjThreads / cgroups);
+      const int cg = tid % cgroups, rl = tid / cgroups;
+      float acc[kProjB][V];
+#pragma unroll
+      for (int bb = 0; bb < kProjB; ++bb)
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[bb][e] = 0.f;
+      if (rl < lanes) {
+        const T* col = w_k + (size_t)r0 * N + (size_t)(c0 + cg) * V;
+        int r = rl;
+        for (; r + 3 * lanes < rows; r += 4 * lanes) {
+          const uint4 x0 = *reinterpret_cast<const uint4*>(col + (size_t)r * N);
+          const uint4 x1 = *reinterpret_cast<const uint4*>(col + (size_t)(r + lanes) * N);
+          const uint4 x2 = *reinterpret_cast<const uint4*>(col + (size_t)(r + 2 * lanes) * N);
+          const uint4 x3 = *reinterpret_cast<const uint4*>(col + (size_t)(r + 3 * lanes) * N);
+#pragma unroll
+          for (int bb = 0; bb < kProjB; ++bb) {
+            if (bb < nb) {
+              fma_vec<T>(acc[bb], x0, hb[bb][r]);
+              fma_vec<T>(acc[bb], x1, hb[bb][r + lanes]);
+              fma_vec<T>(acc[bb], x2, hb[bb][r + 2 * lanes]);
+              fma_vec<T>(acc[bb], x3, hb[bb][r + 3 * lanes]);
+            }
+          }
+        }
+        for (; r < rows; r += lanes) {
+          const uint4 x0 = *reinterpret_cast<const uint4*>(col + (size_t)r * N);
+#pragma unroll
+          for (int bb = 0; bb < kProjB; ++bb)
+            if (bb < nb) fma_vec<T>(acc[bb], x0, hb[bb][r]);
+        }
+      }
+      // Sum the row lanes (fixed order) and write this chunk's partial projections.
+      for (int bb = 0; bb < nb; ++bb) {
+#pragma unroll
+        for (int e = 0; e < V; ++e) accs[tid * V + e] = acc[bb][e];
+        __syncthreads();
+        if (tid < cgroups) {
+          float* out = pp + ((size_t)blockIdx.x * B + b0 + bb) * N + (size_t)(c0 + tid) * V;
+#pragma unroll
+          for (int e = 0; e < V; ++e) {
+            float t = 0.f;
+            for (int l = 0; l < lanes; ++l) t += accs[(l * cgroups + tid) * V + e];
+            out[e] = t;
+          }
+        }
+        __syncthreads();
+      }
+    }
+  }
+}
+
+constexpr int kMlpThreads = 512;
 constexpr int kMlpWarps = kMlpThreads / 32;
+constexpr int kGemvRows = 8;       // rows per warp per pass: their loads are issued together
 
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
@@ -103,62 +210,66 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-// y[r] = act(W[r, :] . x + bias[r]) for r in [0, rows): one warp per row.
+// y[r] = act(W[r, :] . x + bias[r]) for r < rows (W row-major fp32, cols % 4 == 0, x in shared
+// memory).  Each warp takes kGemvRows rows per pass; a lane reads float4s at columns
+// 4*lane + 128*k, so all loads of a pass are in flight together.
 template <bool kRelu>
-__device__ void gemv_rows(const float* __restrict__ W, const float* __restrict__ bias,
-                          const float* x, int rows, int cols, float* y) {
+__device__ void gemv_rows(const float* __restrict__ W, const float* __restrict__ bias, const float* x, int rows,
+                          int cols, float* y) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  for (int r = warp; r < rows; r += kMlpWarps) {
-    const float* w = W + (size_t)r * cols;
-    float s = 0.f;
-    for (int c = lane; c < cols; c += 32) s += w[c] * x[c];
-    s = warp_sum(s) + bias[r];
-    if (lane == 0) y[r] = kRelu ? fmaxf(s, 0.f) : s;
+  for (int r = kGemvRows * warp; r < rows; r += kGemvRows * kMlpWarps) {
+    float s[kGemvRows];
+#pragma unroll
+    for (int u = 0; u < kGemvRows; ++u) s[u] = 0.f;
+    for (int c = 4 * lane; c < cols; c += 128) {
+      const float4 xv = *reinterpret_cast<const float4*>(x + c);
+      float4 wv[kGemvRows];
+#pragma unroll
+      for (int u = 0; u < kGemvRows; ++u)
+        wv[u] = r + u < rows ? __ldg(reinterpret_cast<const float4*>(W + (size_t)(r + u) * cols + c))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < kGemvRows; ++u)
+        s[u] += wv[u].x * xv.x + wv[u].y * xv.y + wv[u].z * xv.z + wv[u].w * xv.w;
+    }
+#pragma unroll
+    for (int u = 0; u < kGemvRows; ++u) {
+      const float t = warp_sum(s[u]);
+      if (lane == 0 && r + u < rows) y[r + u] = kRelu ? fmaxf(t + bias[r + u], 0.f) : t + bias[r + u];
+    }
   }
 }
 
-template <typename T>
-__device__ __forceinline__ float to_f(T x);
-template <> __device__ __forceinline__ float to_f<float>(float x) { return x; }
-template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
-
-// grid (H_kv, B).  Dynamic shared memory: hbar [D] + projection partials [kMlpThreads]
-// + p [d] + tau [d] + hidden [4d] + u [4d] + reduction [kMlpWarps].
-template <typename T>
+// grid (H_kv, B): p = sum of the projection partials of head h, then the task MLP,
+// the router MLP on [p; tau], the head's output row and the threshold.
 __global__ void __launch_bounds__(kMlpThreads)
-router_mlp_kernel(const float* __restrict__ hbar, const T* __restrict__ w_k, ea_router_weights w,
-                  int D, int H_kv, int d, int32_t* __restrict__ head_mode, float* __restrict__ logits) {
-  extern __shared__ float sm[];
+router_mlp_kernel(const float* __restrict__ pp, int n_chunks, int B, int H_kv, int d, ea_router_weights w,
+                  int32_t* __restrict__ head_mode, float* __restrict__ logits) {
+  extern __shared__ __align__(16) float sm[];
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  float* hb = sm;                 // [D]
-  float* part = hb + D;           // [kMlpThreads]
-  float* p = part + kMlpThreads;  // [2d]: p then tau (the router MLP input [p; tau])
+  const int N = H_kv * d;
+  float* p = sm;                  // [2d]: p then tau (the router MLP input [p; tau])
   float* tau = p + d;
   float* hid = p + 2 * d;         // [4d]
   float* u = hid + 4 * d;         // [4d]
-  float* red = u + 4 * d;         // [kMlpWarps]
-  for (int i = tid; i < D; i += kMlpThreads) hb[i] = hbar[(size_t)b * D + i];
-  __syncthreads();
-  // Key projection p[c] = sum_i W_k[i, h*d + c] * hbar[i]: column c = tid % d, row lane
-  // tid / d strides over D; consecutive threads read consecutive columns of a row.
-  const int lanes = kMlpThreads / d;
+  float* part = u + 4 * d;        // [kMlpThreads]
+  float* red = part + kMlpThreads;  // [kMlpWarps]
   {
-    const int c = tid % d, rl = tid / d;
-    const T* col = w_k + (size_t)h * d + c;
-    const size_t ld = (size_t)H_kv * d;
-    float s0 = 0.f, s1 = 0.f;
-    int i = rl;
-    for (; i + lanes < D; i += 2 * lanes) {
-      s0 += to_f(col[(size_t)i * ld]) * hb[i];
-      s1 += to_f(col[(size_t)(i + lanes) * ld]) * hb[i + lanes];
+    const int lanes = kMlpThreads / d, c = tid % d, cl = tid / d;
+    const float* src = pp + (size_t)b * N + (size_t)h * d + c;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    int ch = cl;
+    for (; ch + 7 * lanes < n_chunks; ch += 8 * lanes) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc[k] += src[(size_t)(ch + k * lanes) * B * N];
     }
-    if (i < D) s0 += to_f(col[(size_t)i * ld]) * hb[i];
-    part[tid] = s0 + s1;
+    for (; ch < n_chunks; ch += lanes) acc[0] += src[(size_t)ch * B * N];
+    part[tid] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
   }
   __syncthreads();
   if (tid < d) {
     float s = 0.f;
-    for (int rl = 0; rl < lanes; ++rl) s += part[rl * d + tid];
+    for (int l = 0; l < kMlpThreads / d; ++l) s += part[l * d + tid];
     p[tid] = s;
   }
   __syncthreads();
@@ -204,13 +315,18 @@ PoolPlan plan_pool(int B, int S, int D, int n_boundary, int vec) {
 
 }  // namespace
 
-size_t router_workspace_bytes(int B, int S, int D, int n_boundary) {
-  PoolPlan pl = plan_pool(B, S, D, n_boundary, 4);  // f32 plan has the most chunks; splits match
-  PoolPlan pl8 = plan_pool(B, S, D, n_boundary, 8);
-  const int splits = max(pl.n_splits, pl8.n_splits);
-  size_t partial = (size_t)splits * B * D * sizeof(float);
-  size_t hb = (size_t)B * D * sizeof(float);
-  return ((partial + 255) / 256) * 256 + ((hb + 255) / 256) * 256;
+static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Workspace: pooling partial sums [n_splits][B][D], then projection partials
+// [ceil(D/64)][B][H_kv*d].
+static size_t partial_bytes(int B, int S, int D, int n_boundary) {
+  PoolPlan pl4 = plan_pool(B, S, D, n_boundary, 4), pl8 = plan_pool(B, S, D, n_boundary, 8);
+  return align256((size_t)max(pl4.n_splits, pl8.n_splits) * B * D * sizeof(float));
+}
+static size_t proj_bytes(int B, int D, int N) { return align256((size_t)cdiv(D, kProjRows) * B * N * sizeof(float)); }
+
+size_t router_workspace_bytes(int B, int S, int D, int H_kv, int d, int n_boundary) {
+  return partial_bytes(B, S, D, n_boundary) + proj_bytes(B, D, H_kv * d);
 }
 
 ea_status launch_router(const void* hidden, ea_dtype dtype, int B, int S, int D, int H_kv, int d,
@@ -219,29 +335,22 @@ ea_status launch_router(const void* hidden, ea_dtype dtype, int B, int S, int D,
   const int vec = dtype == EA_DT_BF16 ? 8 : 4;
   PoolPlan pl = plan_pool(B, S, D, prm->n_boundary, vec);
   float* partial = reinterpret_cast<float*>(workspace);
-  size_t partial_bytes = (size_t)pl.n_splits * B * D * sizeof(float);
-  float* hbar = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + ((partial_bytes + 255) / 256) * 256);
+  float* pp = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + partial_bytes(B, S, D, prm->n_boundary));
+  const int N = H_kv * d, n_chunks = cdiv(D, kProjRows);
   dim3 g1(pl.n_chunks, pl.n_splits, B);
-  if (dtype == EA_DT_BF16)
+  if (dtype == EA_DT_BF16) {
     pool_partial_kernel<__nv_bfloat16><<<g1, kPoolThreads, 0, st>>>(
         static_cast<const __nv_bfloat16*>(hidden), S, D, pl.n_rows, pl.a_len, pl.b_start, pl.rows_per_split, partial);
-  else
+    project_kernel<__nv_bfloat16><<<n_chunks, kProjThreads, 0, st>>>(
+        partial, pl.n_splits, B, D, 1.0f / (float)pl.n_rows, static_cast<const __nv_bfloat16*>(w->w_k), N, pp);
+  } else {
     pool_partial_kernel<float><<<g1, kPoolThreads, 0, st>>>(
         static_cast<const float*>(hidden), S, D, pl.n_rows, pl.a_len, pl.b_start, pl.rows_per_split, partial);
-  pool_finish_kernel<<<cdiv(B * D, 256), 256, 0, st>>>(partial, pl.n_splits, B, D, 1.0f / (float)pl.n_rows, hbar);
-  const size_t smem = sizeof(float) * ((size_t)D + kMlpThreads + 2 * d + 8 * d + kMlpWarps);
-  dim3 g2(H_kv, B);
-  if (dtype == EA_DT_BF16) {
-    auto k = router_mlp_kernel<__nv_bfloat16>;
-    if (smem > 48 * 1024 && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return EA_ERR_CUDA;
-    k<<<g2, kMlpThreads, smem, st>>>(hbar, static_cast<const __nv_bfloat16*>(w->w_k), *w, D, H_kv, d, head_mode, logits);
-  } else {
-    auto k = router_mlp_kernel<float>;
-    if (smem > 48 * 1024 && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return EA_ERR_CUDA;
-    k<<<g2, kMlpThreads, smem, st>>>(hbar, static_cast<const float*>(w->w_k), *w, D, H_kv, d, head_mode, logits);
+    project_kernel<float><<<n_chunks, kProjThreads, 0, st>>>(
+        partial, pl.n_splits, B, D, 1.0f / (float)pl.n_rows, static_cast<const float*>(w->w_k), N, pp);
   }
+  const size_t smem = sizeof(float) * ((size_t)10 * d + kMlpThreads + kMlpWarps);
+  router_mlp_kernel<<<dim3(H_kv, B), kMlpThreads, smem, st>>>(pp, n_chunks, B, H_kv, d, *w, head_mode, logits);
   return cudaGetLastError() == cudaSuccess ? EA_OK : EA_ERR_CUDA;
 }
 

@@ -63,7 +63,7 @@ extern "C" ea_status ea_router_static_scratch(const void* hidden, ea_dtype dtype
     return EA_ERR_INVALID_ARG;
   if ((size_t)D * sizeof(float) + 12u * d * sizeof(float) > 200u * 1024u) return EA_ERR_UNSUPPORTED;
   // The problem's scratch must fit the fixed array.
-  if (ea::router_workspace_bytes(B, S, D, prm->n_boundary) > kStaticScratchBytes) return EA_ERR_INVALID_ARG;
+  if (ea::router_workspace_bytes(B, S, D, H_kv, d, prm->n_boundary) > kStaticScratchBytes) return EA_ERR_INVALID_ARG;
   void* scratch = nullptr;
   if (ea_status s = scratch_address(&scratch)) return s;
   return ea::launch_router(hidden, dtype, B, S, D, H_kv, d, w, prm, head_mode, logits, scratch,

@@ -49,7 +49,7 @@ def run_router(w, hidden_storage, weights, n_boundary=None):
     nb = w.n_boundary if n_boundary is None else n_boundary
     hm = torch.zeros(w.B, w.H_kv, dtype=torch.int32, device="cuda")
     z = torch.zeros(w.B, w.H_kv, dtype=torch.float32, device="cuda")
-    ws = torch.zeros(abi.ea_router_workspace_size(w.B, w.S, w.D, nb), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(abi.ea_router_workspace_size(w.B, w.S, w.D, w.H_kv, w.d, nb), dtype=torch.uint8, device="cuda")
     abi.ea_router(to_dev(hidden_storage, w.dtype), {k: to_dev(v, w.dtype) for k, v in weights.items()}, hm, ws,
                   nb, logits=z)
     torch.cuda.synchronize()

@@ -34,7 +34,7 @@ def test_workspace_sizes(lib):
     assert abi.ea_attn_workspace_size(1, 32768, 32, 8) == 512 + 8 * 256 * 2 * 16
     assert abi.ea_attn_workspace_size(1, 100, 7, 2) == 0          # H_q not a multiple of H_kv
     assert abi.ea_attn_workspace_size(1, 65536, 28, 4) == 512 + 4 * 512 * 4 * 16
-    n = abi.ea_router_workspace_size(1, 32768, 4096, 100)
+    n = abi.ea_router_workspace_size(1, 32768, 4096, 8, 128, 100)
     assert n > 4096 * 4 and n % 256 == 0
 
 

@@ -34,7 +34,7 @@ def test_matches_workspace_router_twice(name, n_boundary):
     w = wl.WORKLOADS[name]
     hidden = _gpu.to_dev(wl.hidden_states(w), w.dtype)
     weights = {k: _gpu.to_dev(v, w.dtype) for k, v in wl.router_weights(w).items()}
-    ws = torch.zeros(abi.ea_router_workspace_size(w.B, w.S, w.D, n_boundary), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(abi.ea_router_workspace_size(w.B, w.S, w.D, w.H_kv, w.d, n_boundary), dtype=torch.uint8, device="cuda")
     hm_ref = torch.zeros(w.B, w.H_kv, dtype=torch.int32, device="cuda")
     z_ref = torch.zeros(w.B, w.H_kv, dtype=torch.float32, device="cuda")
     abi.ea_router(hidden, weights, hm_ref, ws, n_boundary, logits=z_ref)
@@ -53,7 +53,7 @@ def test_refuses_problems_beyond_the_scratch_array():
     w = abi.RouterWeights(*([fake] * 9))
     prm = abi.RouterParams(100)
     # 64 samples x D = 32768: the pooled states alone need 8 MiB plus partial sums.
-    assert abi.ea_router_workspace_size(64, 1000, 32768, 100) > (8 << 20)
+    assert abi.ea_router_workspace_size(64, 1000, 32768, 8, 128, 100) > (8 << 20)
     st = lib.ea_router_static_scratch(fake, abi.EA_DT_BF16, 64, 1000, 32768, 8, 128, ctypes.byref(w),
                                       ctypes.byref(prm), fake, None, None)
     assert st == abi.EA_ERR_INVALID_ARG
