@@ -193,6 +193,14 @@ EA_API ea_status ea_effective_sparsity(const int32_t* head_mode, const ea_patter
                                 float* omega_msr_per_sample, ea_sparsity_report* report,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* Test hook for the failure path (no counterpart in the paper): the next
+ * `launches` tensor-core attention launches make the MMA thread of their first
+ * CTA wait on a barrier that nothing arrives on.  That bounded wait runs out
+ * (about 2 s), the CTA drains its own copies and MMAs, frees TMEM and exits, and
+ * the workspace status word reads EA_ERR_TIMEOUT; the output of that CTA's work
+ * items is left unwritten.  0 disables the hook (the default). */
+EA_API void ea_debug_inject_stall(int launches);
+
 /* Synchronises `stream`, reads and clears the workspace's device status
  * word: EA_OK, EA_ERR_TIMEOUT or EA_ERR_BAD_LAYOUT. */
 EA_API ea_status ea_workspace_status(void* workspace, void* stream);

@@ -89,6 +89,8 @@ def _lib():
         lib.ea_router_static_scratch.argtypes = [c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                                  POINTER(RouterWeights), POINTER(RouterParams), c_void_p,
                                                  c_void_p, c_void_p]
+        lib.ea_debug_inject_stall.restype = None
+        lib.ea_debug_inject_stall.argtypes = [c_int]
         lib.ea_workspace_status.restype = st
         lib.ea_workspace_status.argtypes = [c_void_p, c_void_p]
         _LIB = lib
@@ -250,6 +252,12 @@ def ea_effective_sparsity(head_mode, pattern: Pattern, B, S, H_q, H_kv, d, works
 def ea_workspace_status(workspace, stream=None) -> int:
     """Reads and clears the workspace status word; returns the ea_status it maps to."""
     return int(_lib().ea_workspace_status(_dev(workspace, "workspace"), _stream(stream)))
+
+
+def ea_debug_inject_stall(launches: int):
+    """Test hook: the next `launches` tensor-core attention launches stall one CTA until
+    its bounded wait runs out, so the timeout path can be exercised (see include/ea.h)."""
+    _lib().ea_debug_inject_stall(int(launches))
 
 
 def ea_status_string(status: int) -> str:

@@ -39,6 +39,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <atomic>
 #include <mutex>
 #include "ea_common.cuh"
 #include "ea_internal.h"
@@ -61,7 +62,7 @@ constexpr uint32_t OFF_BAR = OFF_V + NV * kTileBytes;
 enum : int {
   B_QFULL = 0, B_QEMPTY = 2, B_KFULL = 4, B_KEMPTY = B_KFULL + NK, B_VFULL = B_KEMPTY + NK,
   B_VEMPTY = B_VFULL + NV, B_SFULL = B_VEMPTY + NV, B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2,
-  B_OFULL = B_PVDONE + 2, B_FIN = B_OFULL + 2, N_BAR = B_FIN + 1
+  B_OFULL = B_PVDONE + 2, B_FIN = B_OFULL + 2, B_NEVER = B_FIN + 1, N_BAR = B_NEVER + 1
 };
 constexpr uint32_t OFF_TMEM = OFF_BAR + N_BAR * 8;
 constexpr uint32_t OFF_ABORT = OFF_TMEM + 4;
@@ -102,6 +103,16 @@ __device__ __forceinline__ bool wait_slow(const Ctx& c, uint32_t bar, uint32_t p
 }
 __device__ __forceinline__ bool wait(const Ctx& c, uint32_t bar, uint32_t parity) {
   return mbar_try_wait(bar, parity) || wait_slow(c, bar, parity);
+}
+// Drain wait: also after an abort, wait (bounded) for this CTA's own copies and MMAs.
+__device__ __forceinline__ void wait_drain(const Ctx& c, uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(c.status, kStatusTimeout);
+      return;
+    }
+  }
 }
 
 struct Item {
@@ -245,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o,
                       const int32_t* __restrict__ head_mode, const PatternDev p, int S, int H_q, int H_kv,
-                      const int4* __restrict__ items, uint32_t* __restrict__ hdr) {
+                      const int4* __restrict__ items, uint32_t* __restrict__ hdr, int inject_stall) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -323,15 +334,15 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       // Drain: the last copy armed on every barrier has landed before the CTA exits.
       for (int st = 0; st < NK; ++st) {
         const int uses = k_it / NK + (st < k_it % NK ? 1 : 0);
-        if (uses > 0) wait_slow(c, c.bar(B_KFULL + st), (uses - 1) & 1);
+        if (uses > 0) wait_drain(c, c.bar(B_KFULL + st), (uses - 1) & 1);
       }
       for (int st = 0; st < NV; ++st) {
         const int uses = v_it / NV + (st < v_it % NV ? 1 : 0);
-        if (uses > 0) wait_slow(c, c.bar(B_VFULL + st), (uses - 1) & 1);
+        if (uses > 0) wait_drain(c, c.bar(B_VFULL + st), (uses - 1) & 1);
       }
 #pragma unroll
       for (int s = 0; s < 2; ++s)
-        if (q_use[s] > 0) wait_slow(c, c.bar(B_QFULL + s), (q_use[s] - 1) & 1);
+        if (q_use[s] > 0) wait_drain(c, c.bar(B_QFULL + s), (q_use[s] - 1) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -339,7 +350,8 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       int q_use0 = 0, q_use1 = 0, p_cnt0 = 0, p_cnt1 = 0, pv_cnt0 = 0, pv_cnt1 = 0;
       bool pend0 = false, pend1 = false;
       int k_it = 0, v_it = 0;
-      bool ok = true;
+      // Test hook for the timeout path: CTA 0 first waits on a barrier nothing arrives on.
+      bool ok = !(inject_stall && blockIdx.x == 0) || wait(c, c.bar(B_NEVER), 0);
       for (int it = 0; ok; ++it) {
         const int idx = item_index(it, blockIdx.x, gridDim.x);
         if (idx >= n_items) break;
@@ -381,7 +393,7 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
       }
       commit(c.bar(B_FIN));                       // every MMA issued here has completed
-      wait_slow(c, c.bar(B_FIN), 0);
+      wait_drain(c, c.bar(B_FIN), 0);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax slots
@@ -514,6 +526,8 @@ bool make_map(CUtensorMap* m, const void* ptr, int B, int S, int H) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+std::atomic<int> g_inject_stall_launches{0};
+
 int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -536,10 +550,15 @@ ea_status launch_attn_tc(const void* q, const void* k, const void* v, void* o, c
     return EA_ERR_CUDA;
   char* ws = static_cast<char*>(workspace);
   const size_t items_off = kWsHeader + ((size_t)B * 4 + 255) / 256 * 256;
+  int inject = 0;
+  for (int n = g_inject_stall_launches.load(); n > 0 && !inject;)
+    if (g_inject_stall_launches.compare_exchange_weak(n, n - 1)) inject = 1;
   kern<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), head_mode, pat, S, H_q,
                                            H_kv, reinterpret_cast<const int4*>(ws + items_off),
-                                           reinterpret_cast<uint32_t*>(ws));
+                                           reinterpret_cast<uint32_t*>(ws), inject);
   return cudaGetLastError() == cudaSuccess ? EA_OK : EA_ERR_CUDA;
 }
 
 }  // namespace ea
+
+extern "C" void ea_debug_inject_stall(int launches) { ea::g_inject_stall_launches.store(launches < 0 ? 0 : launches); }

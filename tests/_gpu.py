@@ -64,7 +64,7 @@ def oracle_router(w, hidden_storage, weights, n_boundary=None):
     return oracle.router.router_forward(h32, hw, w.H_kv, w.d, nb)
 
 
-def run_attention(w, q, k, v, head_mode: np.ndarray, pat: wl.Pattern, split=False, rows=None):
+def run_attention(w, q, k, v, head_mode: np.ndarray, pat: wl.Pattern, split=False, rows=None, check_finite=True):
     """Output rows (all, or ``rows``) as float64 numpy, and the workspace status."""
     dq, dk, dv = to_dev(q, w.dtype), to_dev(k, w.dtype), to_dev(v, w.dtype)
     o = torch.full_like(dq, float("nan"))
@@ -78,7 +78,8 @@ def run_attention(w, q, k, v, head_mode: np.ndarray, pat: wl.Pattern, split=Fals
         abi.ea_hybrid_attn_prefill(dq, dk, dv, hm, dpat, o, ws)
     torch.cuda.synchronize()
     status = abi.ea_workspace_status(ws)
-    assert bool(torch.isfinite(o).all()), "non-finite attention output"
+    if check_finite:
+        assert bool(torch.isfinite(o).all()), "non-finite attention output"
     sel = o if rows is None else o[:, torch.as_tensor(rows, device=o.device)]
     return sel.float().cpu().numpy().astype(np.float64), status
 

@@ -18,7 +18,7 @@ def lib():
 
 def test_every_declared_symbol_is_exported(lib):
     names = abi.declared_symbols()
-    assert len(names) == 10
+    assert len(names) == 11
     for n in names:
         assert hasattr(lib, n), n
 
