@@ -63,8 +63,12 @@ typedef enum { EA_DT_F32 = 0, EA_DT_BF16 = 1 } ea_dtype;
 /* Head kinds (attention patterns).  FULL: keys 0..i.  STREAMING: keys j <= i
  * with j < n_sink or i - j < window (sinks and the local window, united).
  * BLOCK_SPARSE: keys j <= i whose block floor(j/block) is listed for the
- * query block floor(i/block). */
-typedef enum { EA_FULL = 0, EA_STREAMING = 1, EA_BLOCK_SPARSE = 2 } ea_kind;
+ * query block floor(i/block).  STREAMING_BLOCKS: streaming at block
+ * granularity (appendix D.1 runs streaming through the block-sparse kernel):
+ * keys j <= i whose block kb = floor(j/block) is a sink block
+ * (kb < ceil(n_sink/block)) or one of the last ceil(window/block) blocks up to
+ * the query's block. */
+typedef enum { EA_FULL = 0, EA_STREAMING = 1, EA_BLOCK_SPARSE = 2, EA_STREAMING_BLOCKS = 3 } ea_kind;
 
 /* Largest H_kv the calls accept (the per-head kind tables travel by value). */
 #define EA_MAX_KV_HEADS 64
@@ -138,7 +142,7 @@ EA_API ea_status ea_router_static_scratch(const void* hidden, ea_dtype dtype, in
 typedef struct {
   int n_sink;                   /* streaming sink tokens (>= 0); pages: 128        */
   int window;                   /* streaming local window incl. the query (>= 1)   */
-  int block;                    /* block-sparse block edge; must be 128 here       */
+  int block;                    /* block edge of BLOCK_SPARSE / STREAMING_BLOCKS; 128 */
   const int32_t* bs_row_ptr;    /* device CSR [B*H_kv*ceil(S/block) + 1]; rows r = */
   const int32_t* bs_col;        /*   (b*H_kv + h)*n_qb + qb; cols sorted, with qb  */
   long long bs_nnz;             /* entries in bs_col (bounds every column read)    */
@@ -158,6 +162,20 @@ EA_API ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void
                                  int B, int S, int H_q, int H_kv, int d,
                                  const int32_t* head_mode, const ea_pattern_params* pattern,
                                  void* o, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Chunked prefill (appendix D.1 "Sparse Inference": long prompts are prefilled
+ * in chunks, 16,384 tokens in the pages).  q and o [B, S_q, H_q, d] hold query
+ * rows q_offset .. q_offset + S_q - 1 of the sequence; k and v [B, S_k, H_kv, d]
+ * hold its keys from position 0 (a cache; rows past q_offset + S_q - 1 are not
+ * read).  Head patterns use sequence positions, and the block layout has
+ * ceil(S_k / block) query blocks per (sample, KV head).  q_offset % 128 == 0 and
+ * q_offset + S_q <= S_k.  Workspace: ea_attn_workspace_size(B, S_q, H_q, H_kv).
+ * Processing a sequence chunk by chunk gives the same result as one
+ * ea_hybrid_attn_prefill over all of it (the same tiles, in the same order). */
+EA_API ea_status ea_hybrid_attn_prefill_chunk(const void* q, const void* k, const void* v, ea_dtype dtype,
+                                              int B, int S_q, int q_offset, int S_k, int H_q, int H_kv, int d,
+                                              const int32_t* head_mode, const ea_pattern_params* pattern,
+                                              void* o, void* workspace, size_t workspace_bytes, void* stream);
 
 /* The two halves of ea_hybrid_attn_prefill, for callers that time or reuse
  * them.  ea_build_schedule reads head_mode and the pattern on the device and

@@ -28,4 +28,4 @@ part is "parity unpinned" (the written form is pinned, its identity with the
 paper's network is not).
 """
 from . import attention, router, sparsity  # noqa: F401
-from .attention import FULL, STREAMING, BLOCK_SPARSE  # noqa: F401
+from .attention import FULL, STREAMING, BLOCK_SPARSE, STREAMING_BLOCKS  # noqa: F401

@@ -10,7 +10,8 @@ Transformers" (paperlayer.ai summary of arXiv 2601.17367v2):
   * section 1 / B.2 "Intra-layer Hybridization": SA is streaming sparse
     attention (attention sinks plus a local window) or block-sparse attention;
     appendix D.1 "Sparse Inference": 128 sink tokens, block size 64 (the
-    block edge is a parameter here);
+    block edge is a parameter here), streaming run through the block-sparse
+    kernel, i.e. at block granularity;
   * section 1 "Introduction": full attention is the quadratic causal softmax
     attention.
 
@@ -22,6 +23,9 @@ h_kv = h_q // G, G = H_q / H_kv, 0-indexed aligned prefill positions):
   FULL:          L(i) = {0..i}
   STREAMING:     L(i) = {j <= i : j < n_sink or i - j < window}
   BLOCK_SPARSE:  L(i) = {j <= i : floor(j/block) listed for (b, h_kv, floor(i/block))}
+  STREAMING_BLOCKS (streaming at block granularity, appendix D.1):
+                 L(i) = {j <= i : floor(j/block) < ceil(n_sink/block)
+                                  or floor(i/block) - floor(j/block) < ceil(window/block)}
 Readings: token-exact sink and window (the window counts i itself), sink and
 window sets are united, never added; the mode -> kind map is per KV head
 (kind_if_dense[h] / kind_if_sparse[h]).
@@ -30,7 +34,7 @@ from __future__ import annotations
 
 import numpy as np
 
-FULL, STREAMING, BLOCK_SPARSE = 0, 1, 2
+FULL, STREAMING, BLOCK_SPARSE, STREAMING_BLOCKS = 0, 1, 2, 3
 
 
 def head_kind(head_mode, b: int, h_kv: int, kind_if_dense, kind_if_sparse) -> int:
@@ -56,6 +60,12 @@ def live_keys(i: int, kind: int, pattern, b: int = 0, h_kv: int = 0, H_kv: int =
         blk = pattern["block"]
         listed = csr_row(pattern, b, h_kv, i // blk, H_kv, S)
         return j[np.isin(j // blk, listed)]
+    if kind == STREAMING_BLOCKS:
+        blk = pattern["block"]
+        sink_blocks = -(-pattern["n_sink"] // blk)
+        local_blocks = -(-pattern["window"] // blk)
+        kb, qb = j // blk, i // blk
+        return j[(kb < sink_blocks) | (qb - kb < local_blocks)]
     raise ValueError(f"unknown head kind {kind}")
 
 

@@ -22,7 +22,7 @@ import math
 
 import numpy as np
 
-from .attention import FULL, STREAMING, BLOCK_SPARSE, head_kind, live_keys, csr_row
+from .attention import FULL, STREAMING, BLOCK_SPARSE, STREAMING_BLOCKS, head_kind, live_keys, csr_row
 
 TILE = 128
 
@@ -62,6 +62,11 @@ def row_live_counts(S, kind, pattern, b=0, h_kv=0, H_kv=1):
             diag = (i[r0:r1] - r0 + 1) if np.any(cols == qb) else 0
             out[r0:r1] = below + diag
         return out
+    if kind == STREAMING_BLOCKS:
+        blk = int(pattern["block"])
+        sb, lb = -(-int(pattern["n_sink"]) // blk), -(-int(pattern["window"]) // blk)
+        local_start = np.maximum(0, i // blk - lb + 1) * blk        # first key of the local blocks
+        return (i - local_start + 1) + np.maximum(0, np.minimum(sb * blk, local_start))
     raise ValueError(kind)
 
 
@@ -87,6 +92,11 @@ def tile_live_counts(S, kind, pattern, b=0, h_kv=0, H_kv=1):
                     k0, k1 = int(c) * blk, min(int(c) * blk + blk - 1, hi_row, S - 1)
                     if k0 <= k1:
                         tiles.update(range(k0 // TILE, k1 // TILE + 1))
+            out[t] = len(tiles)
+        elif kind == STREAMING_BLOCKS:
+            tiles = set()
+            for i in range(r0, r1 + 1):
+                tiles.update(int(j) // TILE for j in live_keys(i, kind, pattern, b, h_kv, H_kv, S))
             out[t] = len(tiles)
         else:
             raise ValueError(kind)

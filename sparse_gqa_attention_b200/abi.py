@@ -77,6 +77,10 @@ def _lib():
                 c_void_p, POINTER(PatternParams), c_void_p, c_void_p, c_size_t, c_void_p]
         lib.ea_hybrid_attn_prefill.restype = st
         lib.ea_hybrid_attn_prefill.argtypes = attn
+        lib.ea_hybrid_attn_prefill_chunk.restype = st
+        lib.ea_hybrid_attn_prefill_chunk.argtypes = [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
+                                                     c_int, c_int, c_int, c_void_p, POINTER(PatternParams), c_void_p,
+                                                     c_void_p, c_size_t, c_void_p]
         lib.ea_attn_scheduled.restype = st
         lib.ea_attn_scheduled.argtypes = attn
         lib.ea_build_schedule.restype = st
@@ -222,6 +226,19 @@ def ea_hybrid_attn_prefill(q, k, v, head_mode, pattern: Pattern, o, workspace, s
     """o[B, S, H_q, d] <- hybrid-head attention of q, k, v under head_mode and pattern."""
     args, keep = _attn_args(q, k, v, head_mode, pattern, o, workspace, stream)
     _check(_lib().ea_hybrid_attn_prefill(*args), "ea_hybrid_attn_prefill")
+
+
+def ea_hybrid_attn_prefill_chunk(q, k, v, head_mode, pattern: Pattern, o, workspace, q_offset: int, stream=None):
+    """Chunked prefill: q, o [B, S_q, H_q, d] are rows q_offset.. of the sequence whose keys
+    are the rows of k, v [B, S_k, H_kv, d] (q_offset % 128 == 0, q_offset + S_q <= S_k)."""
+    B, S_q, H_q, d = q.shape
+    S_k, H_kv = k.shape[1], k.shape[2]
+    p = pattern.c_struct()
+    _check(_lib().ea_hybrid_attn_prefill_chunk(
+        _dev(q, "q"), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype), _dtype_code(q), B, S_q, int(q_offset), S_k, H_q,
+        H_kv, d, _dev(head_mode, "head_mode", torch.int32), ctypes.byref(p), _dev(o, "o", q.dtype),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream)),
+        "ea_hybrid_attn_prefill_chunk")
 
 
 def ea_build_schedule(head_mode, pattern: Pattern, B, S, H_q, H_kv, d, workspace, stream=None):

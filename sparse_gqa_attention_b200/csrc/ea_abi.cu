@@ -21,30 +21,33 @@ bool any_kind(const ea_pattern_params* p, int H_kv, int kind) {
   return false;
 }
 
-// Checks shared by every attention-side call; fills the device pattern block.
-ea_status check_pattern(const int32_t* head_mode, const ea_pattern_params* p, int B, int S, int H_q, int H_kv,
-                        int d, PatternDev* out) {
+// Checks shared by every attention-side call; fills the device pattern block.  The call's
+// S_q query rows are rows q_offset.. of a sequence whose keys are the S_k rows of k and v.
+ea_status check_pattern(const int32_t* head_mode, const ea_pattern_params* p, int B, int S_q, int S_k,
+                        int q_offset, int H_q, int H_kv, int d, PatternDev* out) {
   if (!head_mode || !p || !p->kind_if_dense || !p->kind_if_sparse) return EA_ERR_INVALID_ARG;
-  if (B < 1 || S < 1 || H_kv < 1 || H_q < 1 || H_q % H_kv != 0) return EA_ERR_INVALID_ARG;
+  if (B < 1 || S_q < 1 || H_kv < 1 || H_q < 1 || H_q % H_kv != 0) return EA_ERR_INVALID_ARG;
+  if (q_offset < 0 || q_offset % kTile != 0 || (long long)q_offset + S_q > (long long)S_k) return EA_ERR_INVALID_ARG;
+  const int S = S_k;
   if (H_kv > EA_MAX_KV_HEADS) return EA_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return EA_ERR_UNSUPPORTED;
   if (p->n_sink < 0 || p->window < 1 || p->block < 1) return EA_ERR_INVALID_ARG;
   if (!(p->softmax_scale >= 0.f) || std::isinf(p->softmax_scale)) return EA_ERR_INVALID_ARG;
   for (int h = 0; h < H_kv; ++h) {
     const int a = p->kind_if_dense[h], b = p->kind_if_sparse[h];
-    if (a < EA_FULL || a > EA_BLOCK_SPARSE || b < EA_FULL || b > EA_BLOCK_SPARSE) return EA_ERR_INVALID_ARG;
+    if (a < EA_FULL || a > EA_STREAMING_BLOCKS || b < EA_FULL || b > EA_STREAMING_BLOCKS) return EA_ERR_INVALID_ARG;
   }
   const bool bsa = any_kind(p, H_kv, EA_BLOCK_SPARSE);
-  if (bsa) {
-    if (!p->bs_row_ptr || !p->bs_col || p->bs_nnz < 0) return EA_ERR_INVALID_ARG;
-    if (p->block != kTile) return EA_ERR_UNSUPPORTED;
-  }
+  if (bsa && (!p->bs_row_ptr || !p->bs_col || p->bs_nnz < 0)) return EA_ERR_INVALID_ARG;
+  if ((bsa || any_kind(p, H_kv, EA_STREAMING_BLOCKS)) && p->block != kTile) return EA_ERR_UNSUPPORTED;
   if ((long long)S > (1LL << 30) || (long long)B * S > (1LL << 31)) return EA_ERR_UNSUPPORTED;
   std::memset(out, 0, sizeof(*out));
   out->n_sink = p->n_sink;
   out->window = p->window;
   out->block = p->block;
-  out->n_qt = cdiv(S, kTile);
+  out->n_qt = cdiv(S_q, kTile);
+  out->q_tile0 = q_offset / kTile;
+  out->n_qb = cdiv(S_k, kTile);
   out->row_ptr = bsa ? p->bs_row_ptr : nullptr;
   out->cols = bsa ? p->bs_col : nullptr;
   out->nnz = bsa ? p->bs_nnz : 0;
@@ -105,7 +108,7 @@ size_t ea_attn_workspace_size(int B, int S, int H_q, int H_kv) {
 ea_status ea_build_schedule(const int32_t* head_mode, const ea_pattern_params* pattern, int B, int S, int H_q,
                             int H_kv, int d, void* workspace, size_t workspace_bytes, void* stream) {
   PatternDev pd;
-  if (ea_status s = check_pattern(head_mode, pattern, B, S, H_q, H_kv, d, &pd)) return s;
+  if (ea_status s = check_pattern(head_mode, pattern, B, S, S, 0, H_q, H_kv, d, &pd)) return s;
   if (ea_status s = check_ws(workspace, workspace_bytes, attn_workspace_bytes(B, S, H_q, H_kv))) return s;
   return launch_schedule(head_mode, pd, B, S, H_q, H_kv, workspace, as_stream(stream));
 }
@@ -114,30 +117,46 @@ ea_status ea_attn_scheduled(const void* q, const void* k, const void* v, ea_dtyp
                             int H_kv, int d, const int32_t* head_mode, const ea_pattern_params* pattern, void* o,
                             void* workspace, size_t workspace_bytes, void* stream) {
   PatternDev pd;
-  if (ea_status s = check_pattern(head_mode, pattern, B, S, H_q, H_kv, d, &pd)) return s;
+  if (ea_status s = check_pattern(head_mode, pattern, B, S, S, 0, H_q, H_kv, d, &pd)) return s;
   if (ea_status s = check_attn_data(q, k, v, o, dtype, d)) return s;
   if (ea_status s = check_ws(workspace, workspace_bytes, attn_workspace_bytes(B, S, H_q, H_kv))) return s;
   if (dtype == EA_DT_F32)
     return launch_attn_simt(static_cast<const float*>(q), static_cast<const float*>(k),
-                            static_cast<const float*>(v), static_cast<float*>(o), head_mode, pd, B, S, H_q, H_kv,
+                            static_cast<const float*>(v), static_cast<float*>(o), head_mode, pd, B, S, S, H_q, H_kv,
                             d, as_stream(stream));
-  return launch_attn_tc(q, k, v, o, head_mode, pd, B, S, H_q, H_kv, workspace, as_stream(stream));
+  return launch_attn_tc(q, k, v, o, head_mode, pd, B, S, S, H_q, H_kv, workspace, as_stream(stream));
+}
+
+static ea_status attn_prefill(const void* q, const void* k, const void* v, ea_dtype dtype, int B, int S_q,
+                              int q_offset, int S_k, int H_q, int H_kv, int d, const int32_t* head_mode,
+                              const ea_pattern_params* pattern, void* o, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  PatternDev pd;
+  if (ea_status s = check_pattern(head_mode, pattern, B, S_q, S_k, q_offset, H_q, H_kv, d, &pd)) return s;
+  if (ea_status s = check_attn_data(q, k, v, o, dtype, d)) return s;
+  if (ea_status s = check_ws(workspace, workspace_bytes, attn_workspace_bytes(B, S_q, H_q, H_kv))) return s;
+  // The schedule kernel also checks head_mode and the block layout on the device.
+  if (ea_status s = launch_schedule(head_mode, pd, B, S_q, H_q, H_kv, workspace, as_stream(stream))) return s;
+  if (dtype == EA_DT_BF16)
+    return launch_attn_tc(q, k, v, o, head_mode, pd, B, S_q, S_k, H_q, H_kv, workspace, as_stream(stream));
+  return launch_attn_simt(static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+                          static_cast<float*>(o), head_mode, pd, B, S_q, S_k, H_q, H_kv, d, as_stream(stream));
 }
 
 ea_status ea_hybrid_attn_prefill(const void* q, const void* k, const void* v, ea_dtype dtype, int B, int S,
                                  int H_q, int H_kv, int d, const int32_t* head_mode,
                                  const ea_pattern_params* pattern, void* o, void* workspace,
                                  size_t workspace_bytes, void* stream) {
-  PatternDev pd;
-  if (ea_status s = check_pattern(head_mode, pattern, B, S, H_q, H_kv, d, &pd)) return s;
-  if (ea_status s = check_attn_data(q, k, v, o, dtype, d)) return s;
-  if (ea_status s = check_ws(workspace, workspace_bytes, attn_workspace_bytes(B, S, H_q, H_kv))) return s;
-  // The schedule kernel also checks head_mode and the block layout on the device.
-  if (ea_status s = launch_schedule(head_mode, pd, B, S, H_q, H_kv, workspace, as_stream(stream))) return s;
-  if (dtype == EA_DT_BF16)
-    return launch_attn_tc(q, k, v, o, head_mode, pd, B, S, H_q, H_kv, workspace, as_stream(stream));
-  return launch_attn_simt(static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
-                          static_cast<float*>(o), head_mode, pd, B, S, H_q, H_kv, d, as_stream(stream));
+  return attn_prefill(q, k, v, dtype, B, S, 0, S, H_q, H_kv, d, head_mode, pattern, o, workspace, workspace_bytes,
+                      stream);
+}
+
+ea_status ea_hybrid_attn_prefill_chunk(const void* q, const void* k, const void* v, ea_dtype dtype, int B,
+                                       int S_q, int q_offset, int S_k, int H_q, int H_kv, int d,
+                                       const int32_t* head_mode, const ea_pattern_params* pattern, void* o,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+  return attn_prefill(q, k, v, dtype, B, S_q, q_offset, S_k, H_q, H_kv, d, head_mode, pattern, o, workspace,
+                      workspace_bytes, stream);
 }
 
 ea_status ea_effective_sparsity(const int32_t* head_mode, const ea_pattern_params* pattern, int B, int S, int H_q,
@@ -145,7 +164,7 @@ ea_status ea_effective_sparsity(const int32_t* head_mode, const ea_pattern_param
                                 void* workspace, size_t workspace_bytes, void* stream) {
   PatternDev pd;
   if (!report) return EA_ERR_INVALID_ARG;
-  if (ea_status s = check_pattern(head_mode, pattern, B, S, H_q, H_kv, d, &pd)) return s;
+  if (ea_status s = check_pattern(head_mode, pattern, B, S, S, 0, H_q, H_kv, d, &pd)) return s;
   if (ea_status s = check_ws(workspace, workspace_bytes, attn_workspace_bytes(B, S, H_q, H_kv))) return s;
   cudaStream_t st = as_stream(stream);
   if (ea_status s = launch_sparsity(head_mode, pd, B, S, H_q, H_kv, workspace, st)) return s;

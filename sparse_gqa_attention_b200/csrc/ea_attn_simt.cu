@@ -24,7 +24,10 @@ __device__ __forceinline__ bool simt_tile_live(const PatternDev& p, int kind, in
     if (c0 < p.n_sink) return true;
     return r0 - (c0 + kKeys - 1) < p.window;  // smallest distance i - j over the tile pair
   }
+  if (kind == EA_STREAMING_BLOCKS)   // block == 128: the 64-row tile sits in one query block
+    return c0 / kTile < cdiv(p.n_sink, kTile) || r0 / kTile - c0 / kTile < cdiv(p.window, kTile);
   if (kind == EA_BLOCK_SPARSE) {   // block == 128: 64-row and 64-key tiles sit in one block each
+    // (r0 is a sequence position; chunks start on a multiple of 128)
     long long a, e;
     csr_row(p, H_kv, b, h, r0 / kTile, a, e);
     for (long long x = a; x < e; ++x)
@@ -38,17 +41,19 @@ template <int HD>
 __global__ void __launch_bounds__(kThreads)
 attn_simt_kernel(const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
                  float* __restrict__ o, const int32_t* __restrict__ head_mode, PatternDev p,
-                 int S, int H_q, int H_kv) {
+                 int S, int S_k, int H_q, int H_kv) {
   constexpr int NC = HD / 32;  // output columns per lane
   extern __shared__ float smem[];
   float (*Ks)[HD + 1] = reinterpret_cast<float (*)[HD + 1]>(smem);
   float (*Vs)[HD] = reinterpret_cast<float (*)[HD]>(smem + kKeys * (HD + 1));
   float (*Qs)[HD] = reinterpret_cast<float (*)[HD]>(smem + kKeys * (HD + 1) + kKeys * HD);
+  // r0 / r1: first and last query row of this CTA in the call (q, o); g0 / g1 in the sequence.
   const int r0 = blockIdx.x * kRows, h_q = blockIdx.y, b = blockIdx.z;
   const int G = H_q / H_kv, h = h_q / G;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int kind = head_kind(p, head_mode, H_kv, b, h);
   const int r1 = min(S, r0 + kRows) - 1;
+  const int q0 = p.q_tile0 * kTile, g0 = q0 + r0, g1 = q0 + r1;
   for (int x = threadIdx.x; x < kRows * HD; x += kThreads) {
     const int r = x / HD, c = x % HD;
     Qs[r][c] = (r0 + r < S) ? q[(((size_t)b * S + r0 + r) * H_q + h_q) * HD + c] : 0.f;
@@ -61,20 +66,20 @@ attn_simt_kernel(const float* __restrict__ q, const float* __restrict__ k, const
 #pragma unroll
     for (int c = 0; c < NC; ++c) acc[rr][c] = 0.f;
   }
-  for (int c0 = 0; c0 <= r1; c0 += kKeys) {
-    if (!simt_tile_live(p, kind, H_kv, b, h, r0, r1, c0)) continue;
+  for (int c0 = 0; c0 <= g1; c0 += kKeys) {
+    if (!simt_tile_live(p, kind, H_kv, b, h, g0, g1, c0)) continue;
     __syncthreads();
     for (int x = threadIdx.x; x < kKeys * HD; x += kThreads) {
       const int j = x / HD, c = x % HD;
-      const bool in = c0 + j < S;
-      const size_t off = (((size_t)b * S + c0 + j) * H_kv + h) * HD + c;
+      const bool in = c0 + j < S_k;
+      const size_t off = (((size_t)b * S_k + c0 + j) * H_kv + h) * HD + c;
       Ks[j][c] = in ? k[off] : 0.f;
       Vs[j][c] = in ? v[off] : 0.f;
     }
     __syncthreads();
 #pragma unroll
     for (int rr = 0; rr < kRowsPerWarp; ++rr) {
-      const int rl = warp * kRowsPerWarp + rr, i = r0 + rl;
+      const int rl = warp * kRowsPerWarp + rr, i = g0 + rl;   // query position in the sequence
       float s[2];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
@@ -83,7 +88,7 @@ attn_simt_kernel(const float* __restrict__ q, const float* __restrict__ k, const
 #pragma unroll 16
         for (int c = 0; c < HD; ++c) dot = fmaf(Qs[rl][c], Ks[j][c], dot);
         const int kind_el = (kind == EA_BLOCK_SPARSE) ? EA_FULL : kind;  // block listed: causal only
-        s[u] = (i < S && c0 + j < S && key_live(p, kind_el, i, c0 + j)) ? dot * p.scale : -INFINITY;
+        s[u] = (r0 + rl < S && c0 + j < S_k && key_live(p, kind_el, i, c0 + j)) ? dot * p.scale : -INFINITY;
       }
       float mt = fmaxf(s[0], s[1]);
 #pragma unroll
@@ -120,14 +125,14 @@ attn_simt_kernel(const float* __restrict__ q, const float* __restrict__ k, const
 }  // namespace
 
 ea_status launch_attn_simt(const float* q, const float* k, const float* v, float* o, const int32_t* head_mode,
-                           const PatternDev& pat, int B, int S, int H_q, int H_kv, int d, cudaStream_t st) {
+                           const PatternDev& pat, int B, int S, int S_k, int H_q, int H_kv, int d, cudaStream_t st) {
   dim3 grid(cdiv(S, kRows), H_q, B);
   const size_t smem = sizeof(float) * ((size_t)kKeys * (d + 1) + (size_t)kKeys * d + (size_t)kRows * d);
   auto kern = d == 64 ? attn_simt_kernel<64> : d == 128 ? attn_simt_kernel<128> : nullptr;
   if (!kern) return EA_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return EA_ERR_CUDA;
-  kern<<<grid, kThreads, smem, st>>>(q, k, v, o, head_mode, pat, S, H_q, H_kv);
+  kern<<<grid, kThreads, smem, st>>>(q, k, v, o, head_mode, pat, S, S_k, H_q, H_kv);
   return cudaGetLastError() == cudaSuccess ? EA_OK : EA_ERR_CUDA;
 }
 

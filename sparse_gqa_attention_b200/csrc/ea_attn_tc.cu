@@ -116,7 +116,7 @@ __device__ __forceinline__ void wait_drain(const Ctx& c, uint32_t bar, uint32_t 
 }
 
 struct Item {
-  int b, h, t, pr, kind, n, sink_end, win_lo;
+  int b, h, t, T, pr, kind, n, sink_end, win_lo;   // t: query tile of this call, T: of the sequence
   long long csr_beg;
   bool two;
 };
@@ -130,20 +130,21 @@ __device__ __forceinline__ Item load_item(const int4* items, int idx, const Patt
   const int4 w = items[idx];
   Item I;
   I.b = w.x; I.h = w.y; I.t = w.z; I.pr = w.w;
+  I.T = I.t + p.q_tile0;
   I.kind = head_kind(p, head_mode, H_kv, I.b, I.h);
   I.two = 2 * I.pr + 1 < G;
   I.sink_end = I.win_lo = 0;
   I.csr_beg = 0;
-  if (I.kind == EA_STREAMING) {
-    stream_ranges(p, I.t, I.sink_end, I.win_lo);
-    I.n = I.sink_end + max(0, I.t - I.win_lo + 1);
+  if (is_streaming(I.kind)) {
+    stream_ranges(p, I.kind, I.T, I.sink_end, I.win_lo);
+    I.n = I.sink_end + max(0, I.T - I.win_lo + 1);
   } else if (I.kind == EA_BLOCK_SPARSE) {
     long long a, e;
-    csr_row(p, H_kv, I.b, I.h, I.t, a, e);
+    csr_row(p, H_kv, I.b, I.h, I.T, a, e);
     I.csr_beg = a;
     I.n = (int)(e - a);
   } else {
-    I.n = I.t + 1;
+    I.n = I.T + 1;
   }
   return I;
 }
@@ -313,7 +314,7 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           ++q_use[s];
         }
         for (int jj = 0; jj < I.n && ok; ++jj) {
-          const int ct = max(0, live_tile(p, I.kind, I.t, jj, I.sink_end, I.win_lo, I.csr_beg));
+          const int ct = max(0, live_tile(p, I.kind, I.T, jj, I.sink_end, I.win_lo, I.csr_beg));
           const int ks = k_it % NK, vs = v_it % NV;
           ok = wait(c, c.bar(B_KEMPTY + ks), ((k_it / NK) & 1) ^ 1);
           if (!ok) break;
@@ -408,11 +409,12 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       if (idx >= n_items) break;
       const Item I = load_item(items, idx, p, head_mode, H_kv, G);
       if (I.n == 0 || (s == 1 && !I.two)) continue;
-      const int i = I.t * BM + row;
+      const int i = I.T * BM + row;        // query position in the sequence
+      const int i_out = I.t * BM + row;    // row of q and o in this call
       const int kind_el = I.kind == EA_STREAMING ? EA_STREAMING : EA_FULL;
       float m_ref = -INFINITY, l = 0.f;
       for (int jj = 0; jj < I.n; ++jj) {
-        const int ct = live_tile(p, I.kind, I.t, jj, I.sink_end, I.win_lo, I.csr_beg);
+        const int ct = live_tile(p, I.kind, I.T, jj, I.sink_end, I.win_lo, I.csr_beg);
         ok = wait(c, c.bar(B_SFULL + s), s_cnt & 1);
         ++s_cnt;
         if (!ok) break;
@@ -431,7 +433,7 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         float f;
         if (ct < 0) {
           f = softmax_tile<1>(x, -1, 0, 0, p.scale_log2, m_ref, l, lane_addr + col_s(s));
-        } else if (tile_needs_mask(p, I.kind, I.t, ct)) {
+        } else if (tile_needs_mask(p, I.kind, I.T, ct)) {
           const int lim = i - ct * BN;
           if (kind_el == EA_STREAMING)
             f = softmax_tile<2>(x, lim, p.n_sink - ct * BN, lim - p.window, p.scale_log2, m_ref, l,
@@ -464,13 +466,13 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       fence_after_sync();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const int h_q = I.h * G + 2 * I.pr + s;
-      __nv_bfloat16* orow = o + (((size_t)I.b * S + i) * H_q + h_q) * HD;
+      __nv_bfloat16* orow = o + (((size_t)I.b * S + i_out) * H_q + h_q) * HD;
 #pragma unroll
       for (int q4 = 0; q4 < HD / 32; ++q4) {
         uint32_t r[32];
         tmem_ld32(lane_addr + col_o(s) + 32 * q4, r);
         tmem_ld_wait();
-        if (i < S) {
+        if (i_out < S) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
             uint4 w;
@@ -538,10 +540,10 @@ int sm_count() {
 }  // namespace
 
 ea_status launch_attn_tc(const void* q, const void* k, const void* v, void* o, const int32_t* head_mode,
-                         const PatternDev& pat, int B, int S, int H_q, int H_kv, void* workspace,
+                         const PatternDev& pat, int B, int S, int S_k, int H_q, int H_kv, void* workspace,
                          cudaStream_t st) {
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, B, S, H_q) || !make_map(&mk, k, B, S, H_kv) || !make_map(&mv, v, B, S, H_kv))
+  if (!make_map(&mq, q, B, S, H_q) || !make_map(&mk, k, B, S_k, H_kv) || !make_map(&mv, v, B, S_k, H_kv))
     return EA_ERR_CUDA;
   const long long n_items = (long long)B * H_kv * pat.n_qt * n_pairs(H_q, H_kv);
   const int grid = (int)std::min<long long>(n_items, sm_count());

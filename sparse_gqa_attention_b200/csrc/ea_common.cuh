@@ -1,8 +1,10 @@
 // ea_common.cuh — device-side definitions shared by the schedule builder, the
 // attention kernels and the sparsity counter.
 //
-// Live key tiles per head kind, for a 128-row query tile t (rows 128t..128t+127)
-// and 128-key tiles c (keys 128c..128c+127); the element rules follow section 2
+// Live key tiles per head kind, for a 128-row query tile t (rows 128t..128t+127 of the
+// sequence: t is the global tile index, so a prefill chunk starting at row q_offset
+// uses t = q_offset/128 + local tile) and 128-key tiles c (keys 128c..128c+127); the
+// element rules follow section 2
 // "Hybrid Head Mechanism" and appendix D.1 "Sparse Inference" of "Elastic
 // Attention: Test-time Adaptive Sparsity Ratios for Efficient Transformers":
 //   FULL          tiles 0..t; only the diagonal tile t needs the causal mask.
@@ -11,6 +13,9 @@
 //                 Every enumerated tile holds at least one live pair.
 //   BLOCK_SPARSE  (block == 128) the listed key blocks of CSR row
 //                 (b*H_kv + h)*n_qt + t; the diagonal tile needs the causal mask.
+//   STREAMING_BLOCKS (block == 128) sink tiles 0..ceil(n_sink/128)-1 (at most t),
+//                 then tiles max(0, t - ceil(window/128) + 1)..t; only the diagonal
+//                 tile needs the causal mask.
 #pragma once
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -37,7 +42,9 @@ struct PatternDev {
   int n_sink;
   int window;
   int block;
-  int n_qt;                 // ceil(S / 128)
+  int n_qt;                 // query tiles of this call: ceil(S_q / 128)
+  int q_tile0;              // global index of the call's first query tile (q_offset / 128)
+  int n_qb;                 // CSR rows per (b, h_kv): ceil(S_k / 128)
   const int32_t* row_ptr;
   const int32_t* cols;
   long long nnz;
@@ -54,17 +61,21 @@ __device__ __forceinline__ int head_kind(const PatternDev& p, const int32_t* hea
   return head_mode[b * H_kv + h] != 0 ? p.kind_sparse[h] : p.kind_dense[h];
 }
 
-// Streaming tile ranges of query tile t: [0, sink_end) and [win_lo, t].
-__device__ __forceinline__ void stream_ranges(const PatternDev& p, int t, int& sink_end, int& win_lo) {
+__device__ __forceinline__ bool is_streaming(int kind) { return kind == EA_STREAMING || kind == EA_STREAMING_BLOCKS; }
+
+// Tile ranges of query tile t for the two streaming kinds: [0, sink_end) and [win_lo, t].
+__device__ __forceinline__ void stream_ranges(const PatternDev& p, int kind, int t, int& sink_end, int& win_lo) {
   sink_end = min(cdiv(p.n_sink, kTile), t + 1);
-  int lo = max(0, t * kTile - p.window + 1) / kTile;
+  const int lo = kind == EA_STREAMING_BLOCKS ? max(0, t - cdiv(p.window, kTile) + 1)
+                                             : max(0, t * kTile - p.window + 1) / kTile;
   win_lo = max(lo, sink_end);
 }
 
-// CSR row [beg, end) of (b, h, t), clamped so a malformed row never reads outside bs_col.
+// CSR row [beg, end) of (b, h, global query tile t), clamped so a malformed row never
+// reads outside bs_col.
 __device__ __forceinline__ void csr_row(const PatternDev& p, int H_kv, int b, int h, int t,
                                         long long& beg, long long& end) {
-  long long r = ((long long)b * H_kv + h) * p.n_qt + t;
+  long long r = ((long long)b * H_kv + h) * p.n_qb + t;
   long long a = p.row_ptr[r], e = p.row_ptr[r + 1];
   a = max(0LL, min(a, p.nnz));
   e = max(a, min(e, p.nnz));
@@ -74,9 +85,9 @@ __device__ __forceinline__ void csr_row(const PatternDev& p, int H_kv, int b, in
 
 // Number of live key tiles of query tile t.
 __device__ __forceinline__ int n_live_tiles(const PatternDev& p, int kind, int H_kv, int b, int h, int t) {
-  if (kind == EA_STREAMING) {
+  if (is_streaming(kind)) {
     int se, wl;
-    stream_ranges(p, t, se, wl);
+    stream_ranges(p, kind, t, se, wl);
     return se + max(0, t - wl + 1);
   }
   if (kind == EA_BLOCK_SPARSE) {
@@ -91,7 +102,7 @@ __device__ __forceinline__ int n_live_tiles(const PatternDev& p, int kind, int H
 // heads a listed column outside [0, t] (a malformed layout) maps to -1: skip it.
 __device__ __forceinline__ int live_tile(const PatternDev& p, int kind, int t, int jj,
                                          int sink_end, int win_lo, long long csr_beg) {
-  if (kind == EA_STREAMING) return jj < sink_end ? jj : win_lo + (jj - sink_end);
+  if (is_streaming(kind)) return jj < sink_end ? jj : win_lo + (jj - sink_end);
   if (kind == EA_BLOCK_SPARSE) {
     int c = p.cols[csr_beg + jj];
     return (c >= 0 && c <= t) ? c : -1;
@@ -112,6 +123,8 @@ __device__ __forceinline__ bool tile_needs_mask(const PatternDev& p, int kind, i
 __device__ __forceinline__ bool key_live(const PatternDev& p, int kind, int i, int j) {
   if (j > i) return false;
   if (kind == EA_STREAMING) return j < p.n_sink || i - j < p.window;
+  if (kind == EA_STREAMING_BLOCKS)
+    return j / kTile < cdiv(p.n_sink, kTile) || i / kTile - j / kTile < cdiv(p.window, kTile);
   return true;  // FULL, and BLOCK_SPARSE inside a listed tile (block == tile)
 }
 

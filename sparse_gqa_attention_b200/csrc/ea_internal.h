@@ -19,9 +19,11 @@ ea_status launch_schedule(const int32_t* head_mode, const PatternDev& pat, int B
                           void* workspace, cudaStream_t st);
 ea_status launch_sparsity(const int32_t* head_mode, const PatternDev& pat, int B, int S, int H_q, int H_kv,
                           void* workspace, cudaStream_t st);
+// S: query rows of this call (q and o); S_k: rows of k and v.  pat.q_tile0 * 128 is the
+// position of the first query row in the sequence.
 ea_status launch_attn_simt(const float* q, const float* k, const float* v, float* o, const int32_t* head_mode,
-                           const PatternDev& pat, int B, int S, int H_q, int H_kv, int d, cudaStream_t st);
+                           const PatternDev& pat, int B, int S, int S_k, int H_q, int H_kv, int d, cudaStream_t st);
 ea_status launch_attn_tc(const void* q, const void* k, const void* v, void* o, const int32_t* head_mode,
-                         const PatternDev& pat, int B, int S, int H_q, int H_kv, void* workspace,
+                         const PatternDev& pat, int B, int S, int S_k, int H_q, int H_kv, void* workspace,
                          cudaStream_t st);
 }  // namespace ea

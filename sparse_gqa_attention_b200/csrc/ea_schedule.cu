@@ -50,13 +50,14 @@ schedule_kernel(const int32_t* __restrict__ head_mode, PatternDev p, int H_kv, i
   __syncthreads();
   uint32_t bad = 0;
   for (int x = tid; x < n_items; x += kSchedThreads) {
-    int b, h, t, pr;
-    decode_item(x, np, p.n_qt, H_kv, b, h, t, pr);
+    int b, h, tl, pr;
+    decode_item(x, np, p.n_qt, H_kv, b, h, tl, pr);
+    const int t = tl + p.q_tile0;   // global query tile
     const int m = head_mode[b * H_kv + h];
     if (m != 0 && m != 1) bad |= kStatusBadMode;
     const int kind = head_kind(p, head_mode, H_kv, b, h);
     if (kind == EA_BLOCK_SPARSE && pr == 0) {
-      const long long r = ((long long)b * H_kv + h) * p.n_qt + t;
+      const long long r = ((long long)b * H_kv + h) * p.n_qb + t;
       const long long a0 = p.row_ptr[r], a1 = p.row_ptr[r + 1];
       if (a0 < 0 || a1 < a0 || a1 > p.nnz || a1 == a0) {
         bad |= kStatusBadLayout;
@@ -73,6 +74,7 @@ schedule_kernel(const int32_t* __restrict__ head_mode, PatternDev p, int H_kv, i
     atomicAdd(&bins[item_cost(p, head_mode, H_kv, G, b, h, t, pr, n_bins)], 1);
   }
   if (bad) atomicOr(hdr + kWsStatus / 4, bad);
+  // (items store the local query tile; the attention kernels add q_tile0)
   __syncthreads();
   // Exclusive scan of the bins in descending cost order: bins[c] <- items costing more than c.
   const int chunk = (n_bins + kSchedThreads - 1) / kSchedThreads;
@@ -96,10 +98,10 @@ schedule_kernel(const int32_t* __restrict__ head_mode, PatternDev p, int H_kv, i
   }
   __syncthreads();
   for (int x = tid; x < n_items; x += kSchedThreads) {
-    int b, h, t, pr;
-    decode_item(x, np, p.n_qt, H_kv, b, h, t, pr);
-    const int pos = atomicAdd(&bins[item_cost(p, head_mode, H_kv, G, b, h, t, pr, n_bins)], 1);
-    items[pos] = make_int4(b, h, t, pr);
+    int b, h, tl, pr;
+    decode_item(x, np, p.n_qt, H_kv, b, h, tl, pr);
+    const int pos = atomicAdd(&bins[item_cost(p, head_mode, H_kv, G, b, h, tl + p.q_tile0, pr, n_bins)], 1);
+    items[pos] = make_int4(b, h, tl, pr);
   }
   if (tid == 0) hdr[kWsNItems / 4] = (uint32_t)n_items;
 }
@@ -115,6 +117,9 @@ sparsity_kernel(const int32_t* __restrict__ head_mode, PatternDev p, int S, int 
   if (i < S) {
     if (kind == EA_STREAMING) {
       cnt = min(i + 1, p.window) + max(0, min(p.n_sink, i - p.window + 1));
+    } else if (kind == EA_STREAMING_BLOCKS) {
+      const long long local_start = (long long)max(0, t - cdiv(p.window, kTile) + 1) * kTile;
+      cnt = (i - local_start + 1) + max(0LL, min((long long)cdiv(p.n_sink, kTile) * kTile, local_start));
     } else if (kind == EA_BLOCK_SPARSE) {
       long long a, e;
       csr_row(p, H_kv, b, h, t, a, e);
@@ -160,7 +165,7 @@ ea_status launch_schedule(const int32_t* head_mode, const PatternDev& pat, int B
   const int G = H_q / H_kv, np = n_pairs(H_q, H_kv);
   const long long n_items = (long long)B * H_kv * pat.n_qt * np;
   if (n_items > (1LL << 30)) return EA_ERR_UNSUPPORTED;
-  const int n_bins = min(kMaxBins, 2 * pat.n_qt + 1);
+  const int n_bins = min(kMaxBins, 2 * (pat.n_qt + pat.q_tile0) + 1);
   char* ws = static_cast<char*>(workspace);
   schedule_kernel<<<1, kSchedThreads, 0, st>>>(head_mode, pat, H_kv, G, np, (int)n_items, n_bins,
                                                reinterpret_cast<uint32_t*>(ws),

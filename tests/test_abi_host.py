@@ -18,7 +18,7 @@ def lib():
 
 def test_every_declared_symbol_is_exported(lib):
     names = abi.declared_symbols()
-    assert len(names) == 11
+    assert len(names) == 12
     for n in names:
         assert hasattr(lib, n), n
 
@@ -80,3 +80,15 @@ def test_router_argument_checks(lib):
                          None, ws, 1 << 30, None) == abi.EA_ERR_UNSUPPORTED      # d not in {64, 128}
     assert lib.ea_router(FAKE, abi.EA_DT_F32, 1, 300, 256, 2, 128, ctypes.byref(w), ctypes.byref(prm), FAKE,
                          None, ws, 8, None) == abi.EA_ERR_INVALID_ARG            # workspace too small
+
+
+@pytest.mark.parametrize("q_offset,S_q,S_k,expect", [
+    (64, 100, 1000, abi.EA_ERR_INVALID_ARG),     # chunks start on a multiple of 128
+    (896, 200, 1000, abi.EA_ERR_INVALID_ARG),    # rows past the keys
+    (-128, 100, 1000, abi.EA_ERR_INVALID_ARG),
+])
+def test_chunk_argument_checks(lib, q_offset, S_q, S_k, expect):
+    pp, keep = _pattern(2)
+    st = lib.ea_hybrid_attn_prefill_chunk(FAKE, FAKE, FAKE, abi.EA_DT_BF16, 1, S_q, q_offset, S_k, 8, 2, 128, FAKE,
+                                          ctypes.byref(pp), FAKE, ctypes.c_void_p(0x100000), 1 << 30, None)
+    assert st == expect

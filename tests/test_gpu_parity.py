@@ -20,9 +20,9 @@ from tests import _gpu
 pytestmark = pytest.mark.gpu
 
 SMALL = ["tiny-fp32-s512", "small-mixed-g4-s1000", "small-bsa-g7-s777", "small-stream-g1-s700",
-         "small-fp32-d128-s300"]
+         "small-fp32-d128-s300", "small-blockstream-g4-s900", "small-fp32-blockstream-s400"]
 FULL = ["llama3-8b-s32k-streaming", "qwen-g7-s64k-blocksparse", "llama3-8b-b4-s16k-mixed",
-        "llama3-8b-s128k-sweep"]
+        "llama3-8b-s128k-sweep", "llama3-8b-s32k-blockstream"]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -92,6 +92,9 @@ EDGE = [  # (S, H_q, H_kv, n_sink, window, sparse kinds, dtype)
     (1, 4, 2, 0, 1, (1, 2), "f32"),
     (129, 3, 1, 2, 70, (1,), "f32"),
     (200, 4, 2, 64, 1, (1, 2), "f32"),
+    (700, 4, 2, 0, 1, (3, 2), "bf16"),
+    (513, 6, 3, 129, 300, (3, 3, 1), "bf16"),
+    (260, 4, 2, 1, 128, (3, 0), "f32"),
 ]
 
 

@@ -197,3 +197,31 @@ def test_sampled_rows_match_all_rows(rng):
     np.testing.assert_array_equal(oa.hybrid_attention_rows(q, k, v, mode, p, rows), full[:, rows])
     sub = oa.hybrid_attention_rows(q[:, rows], k, v, mode, p, rows, q_row_index=rows)
     np.testing.assert_array_equal(sub, full[:, rows])
+
+
+@pytest.mark.parametrize("n_sink,window,block,S", [(128, 256, 64, 300), (1, 1, 16, 77), (0, 1, 8, 50),
+                                                   (20, 40, 16, 100), (0, 10_000, 32, 90)])
+def test_block_streaming_equals_kron_mask_sdpa(rng, n_sink, window, block, S):
+    """Block-granular streaming: sink blocks and local blocks of the block bitmap, made causal."""
+    B, H_kv, G, d = 1, 2, 2, 8
+    q, k, v = _qkv(rng, B, S, G * H_kv, H_kv, d)
+    p = _pattern(H_kv, oa.STREAMING_BLOCKS, n_sink, window, block=block)
+    o = oa.hybrid_attention(q, k, v, np.ones((B, H_kv), np.int32), p)
+    n_qb = -(-S // block)
+    sb, lb = -(-n_sink // block), -(-window // block)
+    rows = [[c for c in range(qb + 1) if c < sb or qb - c < lb] for qb in range(n_qb)]
+    np.testing.assert_allclose(o, _ref.sdpa(q, k, v, mask=_ref.block_mask(S, block, rows)), rtol=0, atol=1e-12)
+
+
+def test_block_streaming_special_cases(rng):
+    B, S, H_kv, d, blk = 1, 70, 1, 8, 16
+    q, k, v = _qkv(rng, B, S, 2, H_kv, d)
+    # no sinks, one local block: block-wise causal attention
+    o = oa.hybrid_attention(q, k, v, np.ones((B, H_kv), np.int32), _pattern(H_kv, oa.STREAMING_BLOCKS, 0, 1, blk))
+    for r0 in range(0, S, blk):
+        r1 = min(S, r0 + blk)
+        np.testing.assert_allclose(o[:, r0:r1], _ref.sdpa(q[:, r0:r1], k[:, r0:r1], v[:, r0:r1], causal=True),
+                                   rtol=0, atol=1e-12)
+    # a window of whole blocks covering the sequence: full causal attention
+    o = oa.hybrid_attention(q, k, v, np.ones((B, H_kv), np.int32), _pattern(H_kv, oa.STREAMING_BLOCKS, 0, S, blk))
+    np.testing.assert_allclose(o, _ref.sdpa(q, k, v, causal=True), rtol=0, atol=1e-12)

@@ -87,3 +87,15 @@ def test_report_plain_and_interval_counts_agree(rng):
     b = osp.sparsity_report(mode, p, 2, S, 4, H_kv, 128)
     for key in ["live_pairs", "live_tiles", "omega_esr"]:
         assert a[key] == b[key]
+
+
+@pytest.mark.parametrize("S,ns,W,block", [(300, 128, 256, 128), (777, 1, 1, 128), (500, 0, 300, 64),
+                                          (260, 300, 5, 32), (1000, 128, 2048, 128)])
+def test_block_streaming_counts_match_kron_mask(S, ns, W, block):
+    from oracle.attention import STREAMING_BLOCKS
+    p = _p(ns, W, block=block, ks=STREAMING_BLOCKS)
+    sb, lb = -(-ns // block), -(-W // block)
+    n_qb = -(-S // block)
+    m = _ref.block_mask(S, block, [[c for c in range(qb + 1) if c < sb or qb - c < lb] for qb in range(n_qb)])
+    np.testing.assert_array_equal(osp.row_live_counts(S, STREAMING_BLOCKS, p), m.sum(axis=1))
+    np.testing.assert_array_equal(osp.tile_live_counts(S, STREAMING_BLOCKS, p), _mask_tiles_live(m))

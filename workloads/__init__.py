@@ -7,7 +7,7 @@ sparsity counting); the CUDA path and the CPU oracle each compute those on
 their own.
 """
 from .generate import (  # noqa: F401
-    FULL, STREAMING, BLOCK_SPARSE,
+    FULL, STREAMING, BLOCK_SPARSE, STREAMING_BLOCKS,
     WORKLOADS, Workload, Pattern,
     bf16_bits_from_f32, f32_from_bf16_bits,
     attention_inputs, hidden_states, router_weights, block_layout, pattern_for,

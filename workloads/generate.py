@@ -10,7 +10,7 @@ drawn from numpy's PCG64 (``numpy.random.default_rng``) with an explicit seed.
 
 Conventions shared with the C ABI and the oracle (an interface, not code):
   * head kinds: 0 = full causal attention, 1 = streaming (sink + local
-    window), 2 = block-sparse;
+    window), 2 = block-sparse, 3 = streaming at block granularity;
   * head_mode[b, h_kv]: 0 = the router's dense decision, 1 = sparse;
   * q, o: [B, S, H_q, d]; k, v: [B, S, H_kv, d]; hidden: [B, S, D]; all
     row-major.  Query head h_q reads KV head h_q // (H_q // H_kv).
@@ -28,7 +28,7 @@ from typing import Optional, Sequence
 
 import numpy as np
 
-FULL, STREAMING, BLOCK_SPARSE = 0, 1, 2
+FULL, STREAMING, BLOCK_SPARSE, STREAMING_BLOCKS = 0, 1, 2, 3
 
 # Stream ids keep the draws of different tensors independent of each other.
 _SID_Q, _SID_K, _SID_V, _SID_HIDDEN, _SID_WK = 11, 12, 13, 14, 15
@@ -98,6 +98,14 @@ WORKLOADS = {w.name: w for w in [
        (STREAMING,) * 4, ("per_sample", (2,))),
     _w("small-fp32-d128-s300", 2, 300, 256, 4, 2, 128, "f32", 5, 64,
        (STREAMING, BLOCK_SPARSE), ("per_sample", (1, 2)), density=0.5),
+    # Streaming at block granularity (sink and local-window blocks of 128 keys).
+    _w("small-blockstream-g4-s900", 2, 900, 256, 8, 2, 128, "bf16", 128, 256,
+       (STREAMING_BLOCKS, BLOCK_SPARSE), ("per_sample", (1, 2)), density=0.3),
+    _w("small-fp32-blockstream-s400", 1, 400, 256, 4, 2, 64, "f32", 100, 129,
+       (STREAMING_BLOCKS, STREAMING), ("fixed", 1)),
+    _w("llama3-8b-s32k-blockstream", 1, 32768, 4096, 32, 8, 128, "bf16", 128, 2048,
+       (STREAMING_BLOCKS,) * 8, ("fixed", 4),
+       note="the Llama layer with streaming heads at block granularity (1 sink block, 16 local blocks)"),
 ]}
 
 
