@@ -112,6 +112,23 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(values, device="cpu"):
+    """Element-wise max of `values` over all ranks of the process group (identity on one process)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(x) for x in values]
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_tflops(flops_per_rank, world, ms_per_step):
+    """Throughput of all ranks together: every rank processes flops_per_rank per step and
+    the slowest rank's step time bounds the job."""
+    return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -234,19 +251,14 @@ def run_cuda(args):
     # Router pooling over the whole sequence (bandwidth measurement).
     router_full = router_bandwidth(w, hidden, weights, dev, st)
 
-    t_max = ms_total
-    if world > 1:
-        tt = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = float(tt.item())
-        et = torch.tensor([e2e["ms_per_step"]], device=dev, dtype=torch.float64)
-        dist.all_reduce(et, op=dist.ReduceOp.MAX)
-        e2e["ms_per_step"] = float(et.item())
+    t_max, e2e_ms, attn_avg = max_over_ranks([ms_total, e2e["ms_per_step"], statistics.mean(attn_ms)], dev)
+    e2e["ms_per_step"] = e2e_ms
+    e2e["value"] = round(whole_job_tflops(e2e["flops_per_step"], world, e2e_ms), 3)
+    del e2e["flops_per_step"]
     ms_step = t_max / args.steps
     pk = peaks()
-    attn_avg = statistics.mean(attn_ms)
     achieved = live_flops / (attn_avg * 1e-3) / 1e12
-    value = world * live_flops / (ms_step * 1e-3) / 1e12
+    value = whole_job_tflops(live_flops, world, ms_step)
     tokens = w.B * w.S
     if rank == 0:
         line = {
@@ -316,7 +328,7 @@ def e2e_measure(args, w, inp, dev, st, weights, pat, forced, rws, aws):
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / n
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    return {"value": round(rep["live_flops"] / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s", "ms_per_step": ms,
+    return {"value": None, "flops_per_step": rep["live_flops"], "unit": "TFLOP/s", "ms_per_step": ms,
             "steps": n, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(o_host.numel() * o_host.element_size() + 4 * w.B + 32),
             "api": "ea_router + ea_hybrid_attn_prefill + ea_effective_sparsity on pinned host buffers"}
