@@ -18,6 +18,10 @@ Modules:
               Router"; appendix D.1 "Sparse Inference").
   sparsity  — model sparsity ratio and effective sparsity ratio (section 2
               "Sparsity Ratio Computation"; appendix C.1 "Sparsity Assignment").
+  xattention — XAttention block selection feeding the block-sparse heads'
+              layout (section 4 "Evaluation Setting": tau = 0.9; the method
+              restated from Xu et al. 2025, whose agreement with XAttention's
+              own implementation is "parity unpinned").
 
 Inputs are taken as given (bf16 inputs arrive already widened to float) and
 every product and sum runs in float64.  Where the pages leave a step open the
@@ -27,5 +31,5 @@ router's wiring with the paper's trained router, which no page fixes: that
 part is "parity unpinned" (the written form is pinned, its identity with the
 paper's network is not).
 """
-from . import attention, router, sparsity  # noqa: F401
+from . import attention, router, sparsity, xattention  # noqa: F401
 from .attention import FULL, STREAMING, BLOCK_SPARSE, STREAMING_BLOCKS  # noqa: F401
