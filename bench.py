@@ -144,6 +144,13 @@ def make_inputs(w):
                 pattern=wl.pattern_for(w))
 
 
+def data_note(w):
+    s = "synthetic (seeded N(0,1)"
+    if w.pos_amp or w.sink_amp:
+        s += f"; q/k plus a positional component (amplitude {w.pos_amp}) and a sink direction ({w.sink_amp})"
+    return s + "; no dataset, tuned random router)"
+
+
 def to_torch(x, dtype_name):
     import torch
     if dtype_name == "bf16" and x.dtype == np.uint16:
@@ -176,7 +183,13 @@ def run_cuda(args):
     weights = {k: to_torch(v, w.dtype).to(dev) for k, v in inp["weights"].items()}
     q, k, v = (to_torch(x, w.dtype).to(dev) for x in (inp["q"], inp["k"], inp["v"]))
     o = torch.empty_like(q)
-    pat = abi.Pattern.from_workloads(inp["pattern"])
+    xattn = w.layout == "xattn"
+    if xattn:
+        pat = abi.Pattern.for_xattn(w.B, w.S, w.H_kv, w.n_sink, w.window, w.kind_if_dense, w.kind_if_sparse)
+        xws = torch.zeros(abi.ea_xattn_workspace_size(w.B, w.S, w.H_q, w.H_kv, w.stride), dtype=torch.uint8,
+                          device=dev)
+    else:
+        pat = abi.Pattern.from_workloads(inp["pattern"])
     head_mode = torch.zeros(w.B, w.H_kv, dtype=torch.int32, device=dev)
     rws = torch.zeros(abi.ea_router_workspace_size(w.B, w.S, w.D, w.H_kv, w.d, w.n_boundary), dtype=torch.uint8, device=dev)
     aws = torch.zeros(abi.ea_attn_workspace_size(w.B, w.S, w.H_q, w.H_kv), dtype=torch.uint8, device=dev)
@@ -186,8 +199,13 @@ def run_cuda(args):
 
     hm = head_mode if forced is None else forced
 
-    def route_and_schedule():
+    def route():
         abi.ea_router(hidden, weights, head_mode, rws, w.n_boundary)
+
+    def select():
+        abi.ea_xattn_block_select(q, k, hm, pat, xws, w.stride, w.tau)
+
+    def schedule():
         abi.ea_build_schedule(hm, pat, w.B, w.S, w.H_q, w.H_kv, w.d, aws)
 
     def attend():
@@ -195,26 +213,30 @@ def run_cuda(args):
 
     # Eager pass first (kernel attributes are set outside capture), then one CUDA graph per
     # part: a step replays them back to back; events between replays time each part.
-    route_and_schedule(); attend(); torch.cuda.synchronize()
-    g_route, g_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_route):
-        route_and_schedule()
-    with torch.cuda.graph(g_attn):
-        attend()
+    parts = [("router", route)] + ([("xattn_select", select)] if xattn else []) + \
+            [("schedule", schedule), ("attention", attend)]
+    for _, fn in parts:
+        fn()
+    torch.cuda.synchronize()
+    graphs = []
+    for name, fn in parts:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        graphs.append((name, g))
     torch.cuda.synchronize()
 
-    ev = {n: [] for n in ("r0", "a1", "a2")}
+    ev = {name: [] for name, _ in parts}
     report = {}
 
     def step(record):
-        if record:
-            e = torch.cuda.Event(enable_timing=True); e.record(st); ev["r0"].append(e)
-        g_route.replay()
-        if record:
-            e = torch.cuda.Event(enable_timing=True); e.record(st); ev["a1"].append(e)
-        g_attn.replay()
-        if record:
-            e = torch.cuda.Event(enable_timing=True); e.record(st); ev["a2"].append(e)
+        for name, g in graphs:
+            if record:
+                a = torch.cuda.Event(enable_timing=True); a.record(st)
+            g.replay()
+            if record:
+                b = torch.cuda.Event(enable_timing=True); b.record(st)
+                ev[name].append((a, b))
         per, rep = abi.ea_effective_sparsity(hm, pat, w.B, w.S, w.H_q, w.H_kv, w.d, aws)   # synchronises
         report["per"], report["rep"] = per, rep
 
@@ -237,17 +259,33 @@ def run_cuda(args):
         if world > 1:
             dist.barrier()
     ms_total = t0.elapsed_time(t1)
-    status = abi.ea_workspace_status(aws)
-    if status != abi.EA_OK:
-        raise RuntimeError(f"device status after the timed steps: {abi.ea_status_string(status)}")
-    attn_ms = [a.elapsed_time(b) for a, b in zip(ev["a1"], ev["a2"])]
-    route_ms = [a.elapsed_time(b) for a, b in zip(ev["r0"], ev["a1"])]
+    for ws_, what in [(aws, "attention")] + ([(xws, "xattn")] if xattn else []):
+        status = abi.ea_workspace_status(ws_)
+        if status != abi.EA_OK:
+            raise RuntimeError(f"device status after the timed steps ({what}): {abi.ea_status_string(status)}")
+    part_ms = {name: statistics.mean(a.elapsed_time(b) for a, b in ev[name]) for name, _ in parts}
+    attn_ms = [a.elapsed_time(b) for a, b in ev["attention"]]
     rep = report["rep"]
     live_flops = rep["live_flops"]
+    xattn_line = None
+    if xattn:
+        mode_h = hm.cpu().numpy()
+        kinds = [[(w.kind_if_sparse[h] if mode_h[b, h] else w.kind_if_dense[h]) for h in range(w.H_kv)]
+                 for b in range(w.B)]
+        live_heads = sum(kind == wl.BLOCK_SPARSE for row in kinds for kind in row) * w.G
+        n_rt = -(-(w.S // w.stride) // 128)
+        x_flops = live_heads * 2.0 * 128 * 128 * (w.stride * w.d) * n_rt * (n_rt + 1) / 2
+        x_ach = x_flops / (part_ms["xattn_select"] * 1e-3) / 1e12
+        pk0 = peaks()
+        xattn_line = {"bound": "tensor", "kernel": "xattn_score_kernel (whole ea_xattn_block_select call)",
+                      "achieved": round(x_ach, 2), "peak": pk0["bf16"], "unit": "TFLOP/s",
+                      "frac": round(x_ach / pk0["bf16"], 4), "flops": x_flops, "stride": w.stride, "tau": w.tau,
+                      "live_query_heads": int(live_heads),
+                      "layout_nnz": int(pat.row_ptr[-1].item())}
 
     # End to end through the same ABI: pinned host inputs -> device, step, result -> host.
-    del g_route, g_attn
-    e2e = e2e_measure(args, w, inp, dev, st, weights, pat, forced, rws, aws, o)
+    del graphs
+    e2e = e2e_measure(args, w, inp, dev, st, weights, pat, forced, rws, aws, o, xws if xattn else None)
 
     # Router pooling over the whole sequence (bandwidth measurement).
     router_full = router_bandwidth(w, hidden, weights, dev, st)
@@ -265,7 +303,7 @@ def run_cuda(args):
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,1); no dataset, random router)",
+            "vs_baseline": None, "dtype": w.dtype, "data": data_note(w),
             "config": {"workload": w.name, "B": w.B, "S": w.S, "D": w.D, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d,
                        "n_sink": w.n_sink, "window": w.window,
                        "omega_msr": float(np.mean(report["per"])), "omega_esr": round(rep["omega_esr"], 6),
@@ -275,10 +313,9 @@ def run_cuda(args):
             "tokens_per_s": round(world * tokens / (ms_step * 1e-3), 1),
             "tflops_dense_causal_equiv": round(world * 4 * w.d * w.H_q * w.B * w.S * (w.S + 1) / 2
                                                / (ms_step * 1e-3) / 1e12, 2),
-            "kernels_ms": {"router+schedule": round(statistics.mean(route_ms), 4),
-                           "attention": round(attn_avg, 4),
-                           "report+sync": round(ms_step - statistics.mean(route_ms) - attn_avg, 4)},
-            "cuda_graphs": "router+schedule and attention captured once, replayed per step",
+            "kernels_ms": dict({n: round(t, 4) for n, t in part_ms.items()},
+                               **{"report+sync": round(ms_step - sum(part_ms.values()), 4)}),
+            "cuda_graphs": " / ".join(n for n, _ in parts) + ": one graph each, captured once, replayed per step",
             "roofline": {"bound": "tensor", "kernel": "hybrid_attn_tc_kernel", "achieved": round(achieved, 2),
                          "peak": pk["bf16"], "unit": "TFLOP/s", "frac": round(achieved / pk["bf16"], 4),
                          "peak_source": f"bf16_tflops burst, {pk['source']}",
@@ -286,8 +323,9 @@ def run_cuda(args):
                          "traffic": ATTN_TRAFFIC.get(attn_source_hash(), {}).get(w.name),
                          "algorithmic_bytes": int(2 * w.B * w.S * w.d * (2 * w.H_q + 2 * w.H_kv))},
             "router_roofline": router_full,
+            **({"xattn_roofline": xattn_line} if xattn_line else {}),
             "e2e": e2e,
-            "gpu_launches": 6 * args.steps,
+            "gpu_launches": (11 if xattn else 6) * args.steps,
             "clocks": clk.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -298,20 +336,23 @@ def run_cuda(args):
         dist.destroy_process_group()
 
 
-def e2e_measure(args, w, inp, dev, st, weights, pat, forced, rws, aws, o_dev, n_chunks=8):
+def e2e_measure(args, w, inp, dev, st, weights, pat, forced, rws, aws, o_dev, xws=None, n_chunks=8):
     """The step end to end through the public API from pinned host buffers.
 
     Every step copies all of hidden, q, k and v host -> device and the output (and the report)
     device -> host.  The copies are pipelined with the compute: the router's pooled rows go
     first, then q/k/v chunk by chunk on an H2D stream while earlier chunks run
     (ea_hybrid_attn_prefill_chunk) and finished chunks' outputs return on a D2H stream; the rest
-    of hidden follows the last chunk.  The timed region spans first copy to last copy."""
+    of hidden follows the last chunk.  With XAttention block selection (xws given) all of q and
+    k land before the selection runs, and only v and o are pipelined.  The timed region spans
+    first copy to last copy."""
     import torch
     from sparse_gqa_attention_b200 import abi
     host = {n: to_torch(inp[n], w.dtype).pin_memory() for n in ("hidden", "q", "k", "v")}
     hid_d = torch.empty_like(host["hidden"], device=dev)
     k_d = torch.empty_like(host["k"], device=dev)
     v_d = torch.empty_like(host["v"], device=dev)
+    q_full = torch.empty_like(host["q"], device=dev) if xws is not None else None
     rows = max(128, (w.S // n_chunks + 127) // 128 * 128)
     bounds = [(r0, min(w.S, r0 + rows)) for r0 in range(0, w.S, rows)]
     q_c = [torch.empty((w.B, r1 - r0, w.H_q, w.d), dtype=host["q"].dtype, device=dev) for r0, r1 in bounds]
@@ -338,16 +379,26 @@ def e2e_measure(args, w, inp, dev, st, weights, pat, forced, rws, aws, o_dev, n_
         ev_pool.record(s_in)
         st.wait_event(ev_pool)
         abi.ea_router(hid_d, weights, head_mode, rws, nb, stream=st)
-        done = []
+        if xws is not None:
+            copy_rows(q_full, host["q"], 0, w.S, s_in)
+            copy_rows(k_d, host["k"], 0, w.S, s_in)
+            ev_qk = torch.cuda.Event()
+            ev_qk.record(s_in)
+            st.wait_event(ev_qk)
+            abi.ea_xattn_block_select(q_full, k_d, hm, pat, xws, w.stride, w.tau, stream=st)
         for c, (r0, r1) in enumerate(bounds):
-            with torch.cuda.stream(s_in):
-                for b in range(w.B):
-                    q_c[c][b].copy_(host["q"][b, r0:r1], non_blocking=True)
-            copy_rows(k_d, host["k"], r0, r1, s_in)
+            if xws is None:
+                with torch.cuda.stream(s_in):
+                    for b in range(w.B):
+                        q_c[c][b].copy_(host["q"][b, r0:r1], non_blocking=True)
+                copy_rows(k_d, host["k"], r0, r1, s_in)
             copy_rows(v_d, host["v"], r0, r1, s_in)
             ev_in = torch.cuda.Event()
             ev_in.record(s_in)
             st.wait_event(ev_in)
+            if xws is not None:
+                with torch.cuda.stream(st):
+                    q_c[c].copy_(q_full[:, r0:r1], non_blocking=True)       # device to device
             abi.ea_hybrid_attn_prefill_chunk(q_c[c], k_d, v_d, hm, pat, o_c[c], ws_c[c], r0, stream=st)
             ev_c = torch.cuda.Event()
             ev_c.record(st)
@@ -355,7 +406,6 @@ def e2e_measure(args, w, inp, dev, st, weights, pat, forced, rws, aws, o_dev, n_
             with torch.cuda.stream(s_out):
                 for b in range(w.B):
                     o_host[b, r0:r1].copy_(o_c[c][b], non_blocking=True)
-            done.append(ev_c)
         for r0, r1 in rest:                      # hidden rows the router does not pool
             copy_rows(hid_d, host["hidden"], r0, r1, s_in)
         per, rep = abi.ea_effective_sparsity(hm, pat, w.B, w.S, w.H_q, w.H_kv, w.d, aws, stream=st)  # synchronises st
@@ -372,18 +422,19 @@ def e2e_measure(args, w, inp, dev, st, weights, pat, forced, rws, aws, o_dev, n_
         rep = step()
     torch.cuda.synchronize()
     ms = (time.perf_counter() - t0) * 1e3 / n
-    for wsc in ws_c:
+    for wsc in ws_c + ([xws] if xws is not None else []):
         if abi.ea_workspace_status(wsc) != abi.EA_OK:
             raise RuntimeError("device status after the end-to-end steps")
     # The chunked calls reproduce the one-launch output bit for bit (same tiles, same order).
     if not torch.equal(o_host, o_dev.cpu()):
         raise RuntimeError("end-to-end output differs from the device-resident step's output")
     h2d = sum(t.numel() * t.element_size() for t in host.values())
+    api = "ea_router + " + ("ea_xattn_block_select + " if xws is not None else "") + \
+        f"ea_hybrid_attn_prefill_chunk x{len(bounds)} + ea_effective_sparsity"
     return {"value": None, "flops_per_step": rep["live_flops"], "unit": "TFLOP/s", "ms_per_step": ms,
             "steps": n, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(o_host.numel() * o_host.element_size() + 4 * w.B + 32),
-            "api": f"ea_router + ea_hybrid_attn_prefill_chunk x{len(bounds)} + ea_effective_sparsity; "
-                   "pinned host buffers, H2D / compute / D2H on separate streams",
+            "api": api + "; pinned host buffers, H2D / compute / D2H on separate streams",
             "timing": "host clock around synchronised steps (first copy issued to last copy done)",
             "output_check": "bitwise equal to the device-resident step"}
 
@@ -430,8 +481,11 @@ def oracle_sample(w, inp, budget_s):
     """Time the oracle on a bounded sample: the router in full (boundary pooling)
     plus attention rows of every query head until ~budget_s of CPU time; the
     rows are spread evenly over the sequence so the per-row cost is
-    representative.  Returns (seconds for the full workload, extrapolated, and
-    the sample description)."""
+    representative.  For XAttention workloads the oracle also selects the block
+    rows of the sampled query blocks (every block-sparse head), and the attention
+    rows read that selection.  Returns (seconds for the full workload,
+    extrapolated, the sample description, and for XAttention workloads the
+    live-tile FLOPs the sampled selections imply)."""
     import oracle
     import workloads as wl
     f64 = lambda x: (wl.f32_from_bf16_bits(x) if x.dtype == np.uint16 else x).astype(np.float64)  # noqa: E731
@@ -445,10 +499,42 @@ def oracle_sample(w, inp, budget_s):
     pd = dict(n_sink=pat.n_sink, window=pat.window, block=pat.block, row_ptr=pat.row_ptr, cols=pat.cols,
               kind_if_dense=pat.kind_if_dense, kind_if_sparse=pat.kind_if_sparse)
     k64, v64 = f64(inp["k"]), f64(inp["v"])
+    xattn = w.layout == "xattn"
+    n_qb = -(-w.S // 128)
+    bs_heads = [(b, h) for b in range(w.B) for h in range(w.H_kv)
+                if (w.kind_if_sparse[h] if mode[b, h] else w.kind_if_dense[h]) == wl.BLOCK_SPARSE]
+    sel = {}                                  # (b, h, qb) -> kept key blocks (oracle selection)
+    t_sel = 0.0
+
+    def select_rows(qbs):
+        nonlocal t_sel
+        t1 = time.perf_counter()
+        for qb in qbs:
+            lo, hi = qb * 128, min((qb + 1) * 128, w.S)
+            for b, h in bs_heads:
+                if (b, h, qb) in sel:
+                    continue
+                a = oracle.xattention.row_importance(f64(inp["q"][b:b + 1, lo:hi]), k64[b:b + 1, :hi], 0, h, qb,
+                                                     w.stride, 128, q_first_row=lo)
+                sel[(b, h, qb)] = oracle.xattention.select_blocks(a, qb, w.tau)
+        t_sel += time.perf_counter() - t1
+
+    def layout():
+        rp, cols = [0], []
+        for b in range(w.B):
+            for h in range(w.H_kv):
+                for qb in range(n_qb):
+                    cols.extend(sel.get((b, h, qb), [qb]))
+                    rp.append(len(cols))
+        return np.array(rp, np.int64), np.array(cols, np.int64)
+
     rows_done, t_attn, n_rows = 0, 0.0, 4
-    while t_attn < budget_s and rows_done < w.S:
+    while t_attn + t_sel < budget_s and rows_done < w.S:
         rows = np.unique(np.linspace(0, w.S - 1, n_rows).astype(np.int64) + rows_done % 7)
         rows = rows[rows < w.S]
+        if xattn:
+            select_rows(np.unique(rows // 128))
+            pd["row_ptr"], pd["cols"] = layout()
         t1 = time.perf_counter()
         oracle.attention.hybrid_attention_rows(f64(inp["q"][:, rows]), k64, v64, mode, pd, rows, q_row_index=rows)
         t_attn += time.perf_counter() - t1
@@ -458,11 +544,30 @@ def oracle_sample(w, inp, budget_s):
     total = t_router + per_row * w.S
     sample = (f"router in full + attention on {rows_done} row positions (all {w.B}x{w.H_q} heads, spread over "
               f"S={w.S}); full-workload time extrapolated as router + per-row time x S")
-    return total, sample
+    live_flops = None
+    if xattn:
+        qbs_done = sorted({qb for (_, _, qb) in sel})
+        total += t_sel / max(1, len(qbs_done)) * n_qb
+        sample += (f"; XAttention selection of {len(qbs_done)} query blocks of the {len(bs_heads)} block-sparse "
+                   f"KV heads, extrapolated x {n_qb} blocks")
+        # live tiles: full heads exactly, block-sparse heads at the sampled mean kept blocks per query block
+        G = w.H_q // w.H_kv
+        tiles = 0.0
+        for b in range(w.B):
+            for h in range(w.H_kv):
+                kind = w.kind_if_sparse[h] if mode[b, h] else w.kind_if_dense[h]
+                rows_t = oracle.sparsity.tile_live_counts(w.S, kind, pd) if kind != wl.BLOCK_SPARSE else None
+                if rows_t is not None:
+                    tiles += G * float(np.sum(rows_t))
+                else:
+                    fr = np.mean([len(sel[(b, h, qb)]) / (qb + 1) for qb in qbs_done])
+                    tiles += G * fr * n_qb * (n_qb + 1) / 2
+        live_flops = 4.0 * w.d * 128 * 128 * tiles
+    return total, sample, live_flops
 
 
 def cpu_baseline(w, inp, live_flops, budget_s=15.0):
-    total, sample = oracle_sample(w, inp, budget_s)
+    total, sample, _ = oracle_sample(w, inp, budget_s)
     return {"value": round(live_flops / total / 1e12, 8), "unit": "TFLOP/s", "cores": cpu_threads(),
             "kind": "oracle", "sample": sample, "seconds_extrapolated": round(total, 2)}
 
@@ -494,14 +599,16 @@ def run_reference(args):
     budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
     times, sample = [], ""
     for i in range(args.warmup + args.steps):
-        total, sample = oracle_sample(w, inp, budget)
+        total, sample, x_flops = oracle_sample(w, inp, budget)
+        if x_flops is not None:          # XAttention layout: live tiles from the oracle's sampled selections
+            live_flops = x_flops
         if i >= args.warmup:
             times.append(total)
     sec = statistics.mean(times)
     value = live_flops / sec / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 8), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 1), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1))",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": data_note(w),
             "config": {"workload": w.name, "B": w.B, "S": w.S, "D": w.D, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d},
             "cpu_baseline": {"value": round(value, 8), "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
                              "sample": sample},

@@ -191,6 +191,49 @@ EA_API ea_status ea_attn_scheduled(const void* q, const void* k, const void* v, 
                             void* o, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * XAttention block selection for the BLOCK_SPARSE heads (section 4
+ * "Evaluation Setting": the block-sparse pattern is XAttention at tau = 0.9;
+ * appendix G.2 "Efficiency Results": FA-XA and XA-SSA pairings).  The pages
+ * name the method; the steps are those of Xu et al., "XAttention: Block Sparse
+ * Attention with Antidiagonal Scoring" (2025):
+ *   R[i, j]   = sum_{m<st} q[i*st+m] . k[j*st+st-1-m]       (reduced i, j < S/st)
+ *   P[i, :]   = softmax over j <= i of R[i, j] * scale / st  (scale as below)
+ *   A[qb, kb] = mean over the G query heads of KV head h of the P mass of the
+ *               128 x 128 tile (qb, kb)
+ *   row qb    = {qb} plus blocks in descending A (ties: lower index) while the
+ *               kept mass < tau * sum_kb A[qb, kb]
+ * Rows are computed for every (b, h) whose kind under head_mode is
+ * BLOCK_SPARSE; the other rows are empty.  The output is the CSR the attention
+ * calls read (bs_row_ptr / bs_col with bs_nnz = cols_capacity), written on
+ * `stream` with no host round trip.
+ * ---------------------------------------------------------------------- */
+
+/* Bytes of workspace ea_xattn_block_select needs: per reduced row (S/stride of
+ * them per query head) one float per 128-key block and per 128-row reduced
+ * tile, plus O(B*H_kv*S/128) for the counts and bitmaps. */
+EA_API size_t ea_xattn_workspace_size(int B, int S, int H_q, int H_kv, int stride);
+
+/* q: device [B, S, H_q, 128] bf16, k: device [B, S, H_kv, 128] bf16 (16-byte
+ * aligned).  stride in {4, 8, 16} with S % stride == 0; S <= 262144;
+ * (H_q / H_kv) * 128 / stride <= 1024; 0 <= tau <= 1.  pattern: kinds,
+ * block == 128 and softmax_scale are read; its bs_* fields are ignored.
+ * row_ptr: device int32 [B*H_kv*ceil(S/128) + 1] (written).  cols: device int32
+ * with cols_capacity >= B*H_kv*n_qb*(n_qb+1)/2 entries, n_qb = ceil(S/128)
+ * (the first row_ptr[last] are written, ascending within each row).
+ * block_scores: NULL, or device float [B, H_kv, n_qb, n_qb] receiving A (zero
+ * above the diagonal and on rows of other kinds).  Buffers are the caller's;
+ * nothing is allocated.  Argument errors return before any launch; device-side
+ * errors (bad head_mode values, a wait past ~2 s) are recorded in the
+ * workspace status word (ea_workspace_status).  Calls on one workspace must not
+ * overlap. */
+EA_API ea_status ea_xattn_block_select(const void* q, const void* k, ea_dtype dtype, int B, int S, int H_q,
+                                       int H_kv, int d, const int32_t* head_mode,
+                                       const ea_pattern_params* pattern, int stride, float tau,
+                                       int32_t* row_ptr, int32_t* cols, long long cols_capacity,
+                                       float* block_scores, void* workspace, size_t workspace_bytes,
+                                       void* stream);
+
+/* ------------------------------------------------------------------------
  * Sparsity report (section 2 "Sparsity Ratio Computation"; appendix C.1).
  * Omega_MSR per sample = sparse KV heads / H_kv.  Omega_ESR = 1 - live
  * (query, key) pairs / causal pairs over all samples and query heads.  Tiles

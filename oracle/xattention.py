@@ -103,6 +103,43 @@ def group_importance(q, k, b: int, h_kv: int, stride: int, block: int, scale: fl
     return acc / G
 
 
+def row_importance(q, k, b: int, h_kv: int, qb: int, stride: int, block: int, scale: float | None = None,
+                   q_first_row: int = 0):
+    """A[qb, 0..qb] alone (steps 1-3 restricted to the reduced rows of query block qb, group
+    mean over the G query heads); the same definition as group_importance, for sampled
+    rows of long sequences.  q may hold only rows q_first_row.. of the sequence (it must
+    include the rows of block qb); k holds rows 0.. (at least through block qb)."""
+    H_q, d = q.shape[2], q.shape[3]
+    S = k.shape[1]
+    H_kv = k.shape[2]
+    G = H_q // H_kv
+    sc = (1.0 / np.sqrt(d) if scale is None else scale) / stride
+    r = block // stride
+    n = -(-S // stride)
+    i_lo, i_hi = qb * r, min((qb + 1) * r, n)
+
+    def reduced_rows(x, first, lo, hi):     # sequence rows lo*st .. hi*st-1 of x (row 0 = first), zero past S
+        out = np.zeros(((hi - lo) * stride, d))
+        top = min(hi * stride, S)
+        out[:top - lo * stride] = x[lo * stride - first:top - first]
+        return out.reshape(hi - lo, stride, d)
+
+    A = np.zeros(qb + 1)
+    kk = reduced_rows(np.asarray(k[b, :, h_kv, :], np.float64), 0, 0, i_hi)
+    for g in range(G):
+        qq = reduced_rows(np.asarray(q[b, :, h_kv * G + g, :], np.float64), q_first_row, i_lo, i_hi)
+        R = np.zeros((i_hi - i_lo, i_hi))
+        for m in range(stride):
+            R += qq[:, m, :] @ kk[:, stride - 1 - m, :].T
+        for t, i in enumerate(range(i_lo, i_hi)):
+            s = sc * R[t, :i + 1]
+            e = np.exp(s - s.max())
+            p = e / e.sum()
+            for kb in range(qb + 1):
+                A[kb] += p[kb * r:(kb + 1) * r].sum()
+    return A / G
+
+
 def select_blocks(a_row: np.ndarray, qb: int, tau: float) -> np.ndarray:
     """Step 4 on one row of importances (entries 0..qb).  Returns the kept blocks, ascending."""
     a = np.asarray(a_row[:qb + 1], np.float64)

@@ -93,6 +93,12 @@ def _lib():
         lib.ea_router_static_scratch.argtypes = [c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                                  POINTER(RouterWeights), POINTER(RouterParams), c_void_p,
                                                  c_void_p, c_void_p]
+        lib.ea_xattn_workspace_size.restype = c_size_t
+        lib.ea_xattn_workspace_size.argtypes = [c_int, c_int, c_int, c_int, c_int]
+        lib.ea_xattn_block_select.restype = st
+        lib.ea_xattn_block_select.argtypes = [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p,
+                                              POINTER(PatternParams), c_int, c_float, c_void_p, c_void_p,
+                                              c_longlong, c_void_p, c_void_p, c_size_t, c_void_p]
         lib.ea_debug_inject_stall.restype = None
         lib.ea_debug_inject_stall.argtypes = [c_int]
         lib.ea_workspace_status.restype = st
@@ -146,6 +152,16 @@ class Pattern:
         self.kind_if_dense = np.ascontiguousarray(kind_if_dense, dtype=np.int8)
         self.kind_if_sparse = np.ascontiguousarray(kind_if_sparse, dtype=np.int8)
         self.softmax_scale = float(softmax_scale)
+
+    @classmethod
+    def for_xattn(cls, B, S, H_kv, n_sink, window, kind_if_dense, kind_if_sparse, softmax_scale=0.0,
+                  device="cuda"):
+        """A pattern whose block layout ea_xattn_block_select fills: row_ptr and cols are
+        device buffers of the sizes that call needs (cols at its worst-case capacity)."""
+        n_qb = -(-S // 128)
+        return cls(n_sink, window, 128, np.zeros(B * H_kv * n_qb + 1, np.int32),
+                   np.zeros(xattn_cols_capacity(B, S, H_kv), np.int32), kind_if_dense, kind_if_sparse,
+                   softmax_scale, device)
 
     @classmethod
     def from_workloads(cls, p, device="cuda"):
@@ -251,6 +267,32 @@ def ea_build_schedule(head_mode, pattern: Pattern, B, S, H_q, H_kv, d, workspace
 def ea_attn_scheduled(q, k, v, head_mode, pattern: Pattern, o, workspace, stream=None):
     args, keep = _attn_args(q, k, v, head_mode, pattern, o, workspace, stream)
     _check(_lib().ea_attn_scheduled(*args), "ea_attn_scheduled")
+
+
+def xattn_cols_capacity(B: int, S: int, H_kv: int) -> int:
+    """Entries ea_xattn_block_select may write into cols: every causal block of every row."""
+    n_qb = -(-S // 128)
+    return B * H_kv * n_qb * (n_qb + 1) // 2
+
+
+def ea_xattn_workspace_size(B: int, S: int, H_q: int, H_kv: int, stride: int = 8) -> int:
+    return int(_lib().ea_xattn_workspace_size(B, S, H_q, H_kv, stride))
+
+
+def ea_xattn_block_select(q, k, head_mode, pattern: Pattern, workspace, stride: int = 8, tau: float = 0.9,
+                          block_scores=None, stream=None):
+    """XAttention's block layout for the BLOCK_SPARSE heads, written into pattern.row_ptr and
+    pattern.cols (a Pattern.for_xattn), with block_scores (float [B, H_kv, n_qb, n_qb]) if given."""
+    B, S, H_q, d = q.shape
+    H_kv = k.shape[2]
+    p = pattern.c_struct()
+    sc = c_void_p(0) if block_scores is None else _dev(block_scores, "block_scores", torch.float32)
+    _check(_lib().ea_xattn_block_select(
+        _dev(q, "q"), _dev(k, "k", q.dtype), _dtype_code(q), B, S, H_q, H_kv, d,
+        _dev(head_mode, "head_mode", torch.int32), ctypes.byref(p), int(stride), float(tau),
+        _dev(pattern.row_ptr, "row_ptr", torch.int32), _dev(pattern.cols, "cols", torch.int32),
+        pattern.cols.numel(), sc, _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream)), "ea_xattn_block_select")
 
 
 def ea_effective_sparsity(head_mode, pattern: Pattern, B, S, H_q, H_kv, d, workspace, stream=None):

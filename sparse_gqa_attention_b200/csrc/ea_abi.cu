@@ -202,6 +202,37 @@ ea_status ea_effective_sparsity(const int32_t* head_mode, const ea_pattern_param
   return EA_OK;
 }
 
+size_t ea_xattn_workspace_size(int B, int S, int H_q, int H_kv, int stride) {
+  if (B < 1 || S < 1 || H_q < 1 || H_kv < 1 || H_q % H_kv != 0) return 0;
+  if (!xattn_shape_ok(S, H_q, H_kv, stride)) return 0;
+  return xattn_workspace_bytes(B, S, H_q, H_kv, stride);
+}
+
+ea_status ea_xattn_block_select(const void* q, const void* k, ea_dtype dtype, int B, int S, int H_q, int H_kv, int d,
+                                const int32_t* head_mode, const ea_pattern_params* pattern, int stride, float tau,
+                                int32_t* row_ptr, int32_t* cols, long long cols_capacity, float* block_scores,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !row_ptr || !cols || !pattern) return EA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k)) return EA_ERR_INVALID_ARG;
+  if (!(tau >= 0.f && tau <= 1.f)) return EA_ERR_INVALID_ARG;
+  if (dtype != EA_DT_BF16 && dtype != EA_DT_F32) return EA_ERR_INVALID_ARG;
+  if (dtype != EA_DT_BF16 || d != 128) return EA_ERR_UNSUPPORTED;
+  // The layout being produced stands in for the pattern's own, so the usual checks apply.
+  ea_pattern_params pp = *pattern;
+  pp.bs_row_ptr = row_ptr;
+  pp.bs_col = cols;
+  pp.bs_nnz = cols_capacity;
+  PatternDev pd;
+  if (ea_status s = check_pattern(head_mode, &pp, B, S, S, 0, H_q, H_kv, d, &pd)) return s;
+  if (pp.block != kTile) return EA_ERR_UNSUPPORTED;
+  if (!xattn_shape_ok(S, H_q, H_kv, stride)) return EA_ERR_UNSUPPORTED;
+  const long long n_qb = cdiv(S, kTile);
+  if (cols_capacity < (long long)B * H_kv * n_qb * (n_qb + 1) / 2) return EA_ERR_INVALID_ARG;
+  if (ea_status s = check_ws(workspace, workspace_bytes, xattn_workspace_bytes(B, S, H_q, H_kv, stride))) return s;
+  return launch_xattn(q, k, head_mode, pd, B, S, H_q, H_kv, stride, tau, row_ptr, cols, block_scores, workspace,
+                      as_stream(stream));
+}
+
 ea_status ea_workspace_status(void* workspace, void* stream) {
   if (!workspace) return EA_ERR_INVALID_ARG;
   cudaStream_t st = as_stream(stream);

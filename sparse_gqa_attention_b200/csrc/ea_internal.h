@@ -26,4 +26,11 @@ ea_status launch_attn_simt(const float* q, const float* k, const float* v, float
 ea_status launch_attn_tc(const void* q, const void* k, const void* v, void* o, const int32_t* head_mode,
                          const PatternDev& pat, int B, int S, int S_k, int H_q, int H_kv, void* workspace,
                          cudaStream_t st);
+
+// XAttention block selection (ea_xattn.cu).
+bool xattn_shape_ok(int S, int H_q, int H_kv, int stride);
+size_t xattn_workspace_bytes(int B, int S, int H_q, int H_kv, int stride);
+ea_status launch_xattn(const void* q, const void* k, const int32_t* head_mode, const PatternDev& pd, int B, int S,
+                       int H_q, int H_kv, int stride, float tau, int32_t* row_ptr, int32_t* cols, float* scores,
+                       void* workspace, cudaStream_t st);
 }  // namespace ea

@@ -18,7 +18,7 @@ def lib():
 
 def test_every_declared_symbol_is_exported(lib):
     names = abi.declared_symbols()
-    assert len(names) == 12
+    assert len(names) == 14
     for n in names:
         assert hasattr(lib, n), n
 
@@ -92,3 +92,47 @@ def test_chunk_argument_checks(lib, q_offset, S_q, S_k, expect):
     st = lib.ea_hybrid_attn_prefill_chunk(FAKE, FAKE, FAKE, abi.EA_DT_BF16, 1, S_q, q_offset, S_k, 8, 2, 128, FAKE,
                                           ctypes.byref(pp), FAKE, ctypes.c_void_p(0x100000), 1 << 30, None)
     assert st == expect
+
+
+def _xattn_call(lib, S=1024, H_q=8, H_kv=2, d=128, dtype=None, stride=8, tau=0.9, block=128, cap=None,
+                ws_bytes=1 << 30, kinds=(0, 2)):
+    dense = np.zeros(H_kv, np.int8)
+    sparse = np.array([kinds[1]] * H_kv, np.int8)
+    pp = abi.PatternParams(128, 2048, block, None, None, 0, dense.ctypes.data_as(ctypes.c_void_p),
+                           sparse.ctypes.data_as(ctypes.c_void_p), 0.0)
+    n_qb = -(-S // 128)
+    cap = 1 * H_kv * n_qb * (n_qb + 1) // 2 if cap is None else cap
+    dtype = abi.EA_DT_BF16 if dtype is None else dtype
+    return lib.ea_xattn_block_select(FAKE, FAKE, dtype, 1, S, H_q, H_kv, d, FAKE, ctypes.byref(pp), stride, tau,
+                                     FAKE, FAKE, cap, None, ctypes.c_void_p(0x100000), ws_bytes, None)
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(stride=6), abi.EA_ERR_UNSUPPORTED),
+    (dict(stride=32), abi.EA_ERR_UNSUPPORTED),
+    (dict(S=1001), abi.EA_ERR_UNSUPPORTED),               # S % stride != 0
+    (dict(S=262144 + 128), abi.EA_ERR_UNSUPPORTED),       # more than 2048 query blocks
+    (dict(tau=1.5), abi.EA_ERR_INVALID_ARG),
+    (dict(tau=-0.1), abi.EA_ERR_INVALID_ARG),
+    (dict(dtype=abi.EA_DT_F32), abi.EA_ERR_UNSUPPORTED),
+    (dict(d=64), abi.EA_ERR_UNSUPPORTED),
+    (dict(block=64), abi.EA_ERR_UNSUPPORTED),
+    (dict(cap=10), abi.EA_ERR_INVALID_ARG),
+    (dict(ws_bytes=1024), abi.EA_ERR_INVALID_ARG),
+    (dict(H_q=7), abi.EA_ERR_INVALID_ARG),
+    (dict(H_q=66, H_kv=2, stride=4), abi.EA_ERR_UNSUPPORTED),   # 33 heads x 32 reduced rows per block
+])
+def test_xattn_argument_checks(lib, case, expect):
+    assert _xattn_call(lib, **case) == expect
+
+
+def test_xattn_workspace_size(lib):
+    B, S, H_q, H_kv, st = 1, 65536, 28, 4, 8
+    n_red, n_rt, n_qb = S // st, S // st // 128, S // 128
+    n = abi.ea_xattn_workspace_size(B, S, H_q, H_kv, st)
+    parts = B * H_q * n_red * n_rt * 4 * (1 + st)          # tile maxima + per-block partial sums
+    assert parts < n < parts + 1024 + B * H_kv * n_qb * 4 * (1 + n_qb // 32 + 1) + 1024
+    assert n % 256 == 0
+    assert abi.ea_xattn_workspace_size(B, S, H_q, H_kv, 6) == 0
+    assert abi.ea_xattn_workspace_size(B, 1001, H_q, H_kv, 8) == 0
+    assert abi.xattn_cols_capacity(2, 300, 3) == 2 * 3 * 3 * 4 // 2

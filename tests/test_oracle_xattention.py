@@ -179,6 +179,18 @@ def test_tau_one_layout_gives_full_causal_attention(rng):
     np.testing.assert_allclose(o, _ref.sdpa(q, k, v, causal=True), atol=1e-12)
 
 
+@pytest.mark.parametrize("S,st,blk,G", [(96, 4, 16, 2), (100, 4, 16, 3), (64, 8, 32, 1)])
+def test_row_importance_matches_full_matrix(rng, S, st, blk, G):
+    q = rng.standard_normal((1, S, 2 * G, 8))
+    k = rng.standard_normal((1, S, 2, 8))
+    full = ox.group_importance(q, k, 0, 1, st, blk)
+    for qb in range(full.shape[0]):
+        np.testing.assert_allclose(ox.row_importance(q, k, 0, 1, qb, st, blk), full[qb, :qb + 1], atol=1e-13)
+        lo = qb * blk       # q given as the block's rows only
+        np.testing.assert_allclose(ox.row_importance(q[:, lo:lo + blk], k, 0, 1, qb, st, blk, q_first_row=lo),
+                                   full[qb, :qb + 1], atol=1e-13)
+
+
 # --- planted mistakes must fail a pin -------------------------------------------------------
 
 def _antidiag_pin_holds(rng):

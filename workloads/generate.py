@@ -1,6 +1,9 @@
 """Seeded input generators for the Elastic Attention prefill path.
 
-Everything here is a random draw, a dtype conversion of a draw, or a shape.
+Everything here is a random draw, a dtype conversion of a draw, a shape, or (for
+the workloads that ask for it) a fixed positional component added to the q/k
+draws so that attention concentrates on nearby keys and a few sink keys, as it
+does in trained models.
 The workloads take the shapes of the layers the pages evaluate (Llama-3.1-8B
 and Qwen3 attention layers, 8K-128K contexts; "Elastic Attention:
 Test-time Adaptive Sparsity Ratios for Efficient Transformers", paperlayer.ai
@@ -32,7 +35,7 @@ FULL, STREAMING, BLOCK_SPARSE, STREAMING_BLOCKS = 0, 1, 2, 3
 
 # Stream ids keep the draws of different tensors independent of each other.
 _SID_Q, _SID_K, _SID_V, _SID_HIDDEN, _SID_WK = 11, 12, 13, 14, 15
-_SID_MLP, _SID_ROUTE, _SID_LAYOUT = 16, 17, 18
+_SID_MLP, _SID_ROUTE, _SID_LAYOUT, _SID_SINK = 16, 17, 18, 19
 _ROW_CHUNK = 1024
 
 _TUNING_PATH = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
@@ -59,6 +62,11 @@ class Workload:
     n_boundary: int = 100
     seed: int = 0
     note: str = ""
+    layout: str = "random"          # "random": block_layout(); "xattn": selected by XAttention
+    stride: int = 8                 # XAttention antidiagonal stride
+    tau: float = 0.9                # XAttention threshold
+    pos_amp: float = 0.0            # amplitude of the positional component of q and k
+    sink_amp: float = 0.0           # amplitude of the sink direction (all q rows, the first 4 k rows)
 
     @property
     def G(self) -> int:
@@ -66,11 +74,17 @@ class Workload:
 
 
 def _w(name, B, S, D, H_q, H_kv, d, dtype, n_sink, window, kinds_sparse, routing,
-       block=128, density=0.1, note=""):
+       block=128, density=0.1, note="", kinds_dense=None, **extra):
     return Workload(name=name, B=B, S=S, D=D, H_q=H_q, H_kv=H_kv, d=d, dtype=dtype,
                     n_sink=n_sink, window=window, block=block, density=density,
-                    kind_if_dense=(FULL,) * H_kv, kind_if_sparse=tuple(kinds_sparse),
-                    routing=routing, note=note)
+                    kind_if_dense=(FULL,) * H_kv if kinds_dense is None else tuple(kinds_dense),
+                    kind_if_sparse=tuple(kinds_sparse), routing=routing, note=note, **extra)
+
+
+# Amplitudes: at S = 32k-64k XAttention (stride 8, tau 0.9) then keeps ~5-15 % of the causal blocks,
+# most query blocks only their diagonal and some tens of blocks; the small parity cases use a
+# weaker positional component so that their selections are not all diagonal.
+_XA = dict(layout="xattn", sink_amp=10.0)
 
 
 _ALT = lambda H: tuple(STREAMING if h % 2 == 0 else BLOCK_SPARSE for h in range(H))  # noqa: E731
@@ -106,6 +120,19 @@ WORKLOADS = {w.name: w for w in [
     _w("llama3-8b-s32k-blockstream", 1, 32768, 4096, 32, 8, 128, "bf16", 128, 2048,
        (STREAMING_BLOCKS,) * 8, ("fixed", 4),
        note="the Llama layer with streaming heads at block granularity (1 sink block, 16 local blocks)"),
+    # XAttention block selection feeding the block-sparse heads (q/k with local + sink structure).
+    _w("qwen-g7-s64k-xattn", 1, 65536, 3584, 28, 4, 128, "bf16", 128, 2048, (BLOCK_SPARSE,) * 4,
+       ("fixed", 2), note="FA-XA: dense heads full, sparse heads XAttention (stride 8, tau 0.9)", pos_amp=1.8,
+       **_XA),
+    _w("llama3-8b-s32k-xassa", 1, 32768, 4096, 32, 8, 128, "bf16", 128, 2048, (STREAMING,) * 8,
+       ("fixed", 4), kinds_dense=(BLOCK_SPARSE,) * 8,
+       note="XA-SSA: dense heads XAttention (stride 8, tau 0.9), sparse heads streaming", pos_amp=1.7, **_XA),
+    _w("small-xattn-g4-s2560", 2, 2560, 256, 8, 2, 128, "bf16", 64, 300, (BLOCK_SPARSE,) * 2,
+       ("per_sample", (1, 2)), pos_amp=1.5, **_XA),
+    _w("small-xattn-g7-s1000", 1, 1000, 384, 14, 2, 128, "bf16", 0, 1, (BLOCK_SPARSE,) * 2,
+       ("fixed", 1), pos_amp=1.5, **_XA),
+    _w("small-xassa-g4-s1536", 1, 1536, 256, 8, 2, 128, "bf16", 128, 256, (STREAMING,) * 2,
+       ("fixed", 1), kinds_dense=(BLOCK_SPARSE,) * 2, pos_amp=1.5, **_XA),
 ]}
 
 
@@ -170,16 +197,55 @@ def _row_chunked_normal(seed, sid, b, S, row_shape, rows: Optional[np.ndarray] =
 # attention inputs
 # ---------------------------------------------------------------------------
 
+def positional_component(rows: np.ndarray, d: int) -> np.ndarray:
+    """[len(rows), d] float32: (cos, sin) pairs of the row index at d/2 frequencies whose
+    periods run geometrically from 8 to 1024 positions.  Added to q and k with the same
+    amplitude, it raises q_i . k_j when |i - j| is small (within a few hundred positions)."""
+    rows = np.asarray(rows, np.float64)
+    f = np.arange(d // 2, dtype=np.float64)
+    period = 8.0 * (128.0 ** (f / max(d // 2 - 1, 1)))
+    ang = rows[:, None] * (2.0 * np.pi / period)[None, :]
+    out = np.empty((len(rows), d), np.float64)
+    out[:, 0::2] = np.cos(ang)
+    out[:, 1::2] = np.sin(ang)
+    return out.astype(np.float32)
+
+
+def _sink_direction(w: Workload) -> np.ndarray:
+    v = _rng(w.seed, _SID_SINK).standard_normal(w.d)
+    return (v / np.linalg.norm(v)).astype(np.float32)
+
+
+def _structured(x: np.ndarray, rows: np.ndarray, w: Workload, is_key: bool) -> np.ndarray:
+    """x [n, H, d] plus the positional component (both q and k) and the sink direction (every q
+    row; k rows 0..3)."""
+    if w.pos_amp == 0.0 and w.sink_amp == 0.0:
+        return x
+    out = x + np.float32(w.pos_amp) * positional_component(rows, w.d)[:, None, :]
+    if w.sink_amp != 0.0:
+        s = np.float32(w.sink_amp) * _sink_direction(w)
+        if is_key:
+            out[np.asarray(rows) < 4] += s
+        else:
+            out += s
+    return out
+
+
 def attention_inputs(w: Workload, batches: Optional[Sequence[int]] = None, q_rows=None):
-    """q, k, v ~ N(0,1) in storage form (uint16 bf16 bits, or float32).
+    """q, k, v ~ N(0,1) in storage form (uint16 bf16 bits, or float32); workloads with
+    pos_amp / sink_amp add the structured components of ``_structured`` to q and k.
 
     ``batches`` restricts the draw to some samples (the arrays then hold only
     those); ``q_rows`` restricts q to some rows (k and v stay whole)."""
     bs = list(range(w.B)) if batches is None else list(batches)
+    all_rows = np.arange(w.S)
+    qr = all_rows if q_rows is None else np.asarray(q_rows, np.int64)
     qs, ks, vs = [], [], []
     for b in bs:
-        qs.append(_storage(_row_chunked_normal(w.seed, _SID_Q, b, w.S, (w.H_q, w.d), q_rows), w.dtype))
-        ks.append(_storage(_row_chunked_normal(w.seed, _SID_K, b, w.S, (w.H_kv, w.d)), w.dtype))
+        q = _structured(_row_chunked_normal(w.seed, _SID_Q, b, w.S, (w.H_q, w.d), q_rows), qr, w, False)
+        k = _structured(_row_chunked_normal(w.seed, _SID_K, b, w.S, (w.H_kv, w.d)), all_rows, w, True)
+        qs.append(_storage(q, w.dtype))
+        ks.append(_storage(k, w.dtype))
         vs.append(_storage(_row_chunked_normal(w.seed, _SID_V, b, w.S, (w.H_kv, w.d)), w.dtype))
     return np.stack(qs), np.stack(ks), np.stack(vs)
 
