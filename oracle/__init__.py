@@ -18,6 +18,10 @@ Modules:
               Router"; appendix D.1 "Sparse Inference").
   sparsity  — model sparsity ratio and effective sparsity ratio (section 2
               "Sparsity Ratio Computation"; appendix C.1 "Sparsity Assignment").
+  assignment — retrieval scores, static retrieval-head assignment
+              k = floor((1 - Omega_MSR) L H) and whole-stack sparsity
+              (appendix C.1 "Retrieval Score Calculation", "Sparsity
+              Assignment").
   xattention — XAttention block selection feeding the block-sparse heads'
               layout (section 4 "Evaluation Setting": tau = 0.9; the method
               restated from Xu et al. 2025, whose agreement with XAttention's
@@ -31,5 +35,5 @@ router's wiring with the paper's trained router, which no page fixes: that
 part is "parity unpinned" (the written form is pinned, its identity with the
 paper's network is not).
 """
-from . import attention, router, sparsity, xattention  # noqa: F401
+from . import assignment, attention, router, sparsity, xattention  # noqa: F401
 from .attention import FULL, STREAMING, BLOCK_SPARSE, STREAMING_BLOCKS  # noqa: F401
