@@ -254,6 +254,45 @@ EA_API ea_status ea_effective_sparsity(const int32_t* head_mode, const ea_patter
                                 float* omega_msr_per_sample, ea_sparsity_report* report,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* The same report over a stack of L layers that share `pattern`: head_mode is
+ * device int32 [L, B, H_kv] (layer-major).  Pairs, tiles and FLOPs are summed
+ * over the layers; Omega_ESR = 1 - live / causal pairs of all layers; Omega_MSR
+ * per sample = its sparse KV heads over L * H_kv.  Workspace:
+ * ea_attn_workspace_size(B, S, H_q, H_kv).  Synchronises `stream`. */
+EA_API ea_status ea_model_sparsity(const int32_t* head_mode, const ea_pattern_params* pattern,
+                                   int L, int B, int S, int H_q, int H_kv, int d,
+                                   float* omega_msr_per_sample, ea_sparsity_report* report,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Static retrieval-head assignment (appendix C.1 "Retrieval Score
+ * Calculation" and "Sparsity Assignment").
+ *   score[b, h_q] = sum_{needle_begin <= j < needle_end} softmax_j(scale q_{S-1} . k_j)
+ * (the attention mass of the last token on the needle span), per layer; then
+ *   kv_score[l, h] = mean over b and the G query heads of KV head h of score
+ *   k = floor((1 - omega_msr) * L * H_kv)   (double precision)
+ *   head_mode[l, b, h] = 0 (full) for the k best kv_scores (ties: lower
+ *   l * H_kv + h first), 1 (sparse) for the others, the same for every b.
+ * ---------------------------------------------------------------------- */
+
+/* Bytes of workspace ea_retrieval_scores needs (per-slice partial sums). */
+EA_API size_t ea_retrieval_workspace_size(int B, int S, int H_q);
+
+/* One layer's retrieval scores.  q: device [B, S, H_q, d], k: device
+ * [B, S, H_kv, d] (bf16 or f32, 16-byte aligned; only q row S-1 is read);
+ * d in {64, 128}; 0 <= needle_begin <= needle_end <= S; softmax_scale 0
+ * selects 1/sqrt(d).  scores: device float [B, H_q] (written).  fp32
+ * accumulation. */
+EA_API ea_status ea_retrieval_scores(const void* q, const void* k, ea_dtype dtype, int B, int S, int H_q,
+                                     int H_kv, int d, int needle_begin, int needle_end, float softmax_scale,
+                                     float* scores, void* workspace, size_t workspace_bytes, void* stream);
+
+/* scores: device float [L, B, H_q] (the layers' ea_retrieval_scores outputs
+ * stacked); head_mode: device int32 [L, B, H_kv] (written).  L * H_kv <= 8192,
+ * 0 <= omega_msr <= 1.  One kernel launch, no allocation. */
+EA_API ea_status ea_static_head_assignment(const float* scores, int L, int B, int H_q, int H_kv,
+                                           double omega_msr, int32_t* head_mode, void* stream);
+
 /* Test hook for the failure path (no counterpart in the paper): the next
  * `launches` tensor-core attention launches make the MMA thread of their first
  * CTA wait on a barrier that nothing arrives on.  That bounded wait runs out

@@ -99,6 +99,17 @@ def _lib():
         lib.ea_xattn_block_select.argtypes = [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p,
                                               POINTER(PatternParams), c_int, c_float, c_void_p, c_void_p,
                                               c_longlong, c_void_p, c_void_p, c_size_t, c_void_p]
+        lib.ea_model_sparsity.restype = st
+        lib.ea_model_sparsity.argtypes = [c_void_p, POINTER(PatternParams), c_int, c_int, c_int, c_int, c_int, c_int,
+                                          c_void_p, POINTER(SparsityReport), c_void_p, c_size_t, c_void_p]
+        lib.ea_retrieval_workspace_size.restype = c_size_t
+        lib.ea_retrieval_workspace_size.argtypes = [c_int, c_int, c_int]
+        lib.ea_retrieval_scores.restype = st
+        lib.ea_retrieval_scores.argtypes = [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                            c_int, c_float, c_void_p, c_void_p, c_size_t, c_void_p]
+        lib.ea_static_head_assignment.restype = st
+        lib.ea_static_head_assignment.argtypes = [c_void_p, c_int, c_int, c_int, c_int, c_double, c_void_p,
+                                                  c_void_p]
         lib.ea_debug_inject_stall.restype = None
         lib.ea_debug_inject_stall.argtypes = [c_int]
         lib.ea_workspace_status.restype = st
@@ -307,6 +318,42 @@ def ea_effective_sparsity(head_mode, pattern: Pattern, B, S, H_q, H_kv, d, works
     _check(status, "ea_effective_sparsity")
     return per, {f: getattr(rep, f) for f, _ in SparsityReport._fields_}
 
+
+
+def ea_model_sparsity(head_mode, pattern: Pattern, L, B, S, H_q, H_kv, d, workspace, stream=None):
+    """Whole-stack report for head_mode [L, B, H_kv] (synchronises the stream)."""
+    p = pattern.c_struct()
+    per = (c_float * B)()
+    rep = SparsityReport()
+    _check(_lib().ea_model_sparsity(_dev(head_mode, "head_mode", torch.int32), ctypes.byref(p), L, B, S, H_q, H_kv,
+                                    d, per, ctypes.byref(rep), _dev(workspace, "workspace"),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)),
+           "ea_model_sparsity")
+    return np.array(per[:], np.float64), {f: getattr(rep, f) for f, _ in SparsityReport._fields_}
+
+
+def ea_retrieval_workspace_size(B: int, S: int, H_q: int) -> int:
+    return int(_lib().ea_retrieval_workspace_size(B, S, H_q))
+
+
+def ea_retrieval_scores(q, k, needle_begin: int, needle_end: int, scores, workspace, softmax_scale: float = 0.0,
+                        stream=None):
+    """scores [B, H_q] (float32, device) <- attention mass of the last token on the needle span."""
+    B, S, H_q, d = q.shape
+    H_kv = k.shape[2]
+    _check(_lib().ea_retrieval_scores(_dev(q, "q"), _dev(k, "k", q.dtype), _dtype_code(q), B, S, H_q, H_kv, d,
+                                      int(needle_begin), int(needle_end), float(softmax_scale),
+                                      _dev(scores, "scores", torch.float32), _dev(workspace, "workspace"),
+                                      workspace.numel() * workspace.element_size(), _stream(stream)),
+           "ea_retrieval_scores")
+
+
+def ea_static_head_assignment(scores, H_kv: int, omega_msr: float, head_mode, stream=None):
+    """head_mode [L, B, H_kv] (int32, device) <- static assignment from scores [L, B, H_q]."""
+    L, B, H_q = scores.shape
+    _check(_lib().ea_static_head_assignment(_dev(scores, "scores", torch.float32), L, B, H_q, H_kv,
+                                            float(omega_msr), _dev(head_mode, "head_mode", torch.int32),
+                                            _stream(stream)), "ea_static_head_assignment")
 
 def ea_workspace_status(workspace, stream=None) -> int:
     """Reads and clears the workspace status word; returns the ea_status it maps to."""

@@ -159,15 +159,18 @@ ea_status ea_hybrid_attn_prefill_chunk(const void* q, const void* k, const void*
                       workspace_bytes, stream);
 }
 
-ea_status ea_effective_sparsity(const int32_t* head_mode, const ea_pattern_params* pattern, int B, int S, int H_q,
-                                int H_kv, int d, float* omega_msr_per_sample, ea_sparsity_report* report,
+// Sparsity counts of L layers (head_mode [L, B, H_kv], one pattern) accumulated on the device.
+static ea_status stack_sparsity(const int32_t* head_mode, const ea_pattern_params* pattern, int L, int B, int S,
+                                int H_q, int H_kv, int d, float* omega_msr_per_sample, ea_sparsity_report* report,
                                 void* workspace, size_t workspace_bytes, void* stream) {
   PatternDev pd;
-  if (!report) return EA_ERR_INVALID_ARG;
+  if (!report || L < 1) return EA_ERR_INVALID_ARG;
   if (ea_status s = check_pattern(head_mode, pattern, B, S, S, 0, H_q, H_kv, d, &pd)) return s;
   if (ea_status s = check_ws(workspace, workspace_bytes, attn_workspace_bytes(B, S, H_q, H_kv))) return s;
   cudaStream_t st = as_stream(stream);
-  if (ea_status s = launch_sparsity(head_mode, pd, B, S, H_q, H_kv, workspace, st)) return s;
+  for (int l = 0; l < L; ++l)
+    if (ea_status s = launch_sparsity(head_mode + (size_t)l * B * H_kv, pd, B, S, H_q, H_kv, workspace, st, l == 0))
+      return s;
   char* ws = static_cast<char*>(workspace);
   unsigned long long counters[2] = {0, 0};
   uint32_t status = 0;
@@ -183,23 +186,69 @@ ea_status ea_effective_sparsity(const int32_t* head_mode, const ea_pattern_param
   }
   double mean = 0.0;
   for (int b = 0; b < B; ++b) {
-    const double om = (double)sparse[b] / H_kv;
+    const double om = (double)sparse[b] / ((double)L * H_kv);
     if (omega_msr_per_sample) omega_msr_per_sample[b] = (float)om;
     mean += om / B;
   }
   delete[] sparse;
-  const long long causal_pairs = (long long)B * H_q * ((long long)S * (S + 1) / 2);
+  const long long causal_pairs = (long long)L * B * H_q * ((long long)S * (S + 1) / 2);
   const long long nq = cdiv(S, kTile);
   report->omega_msr_mean = mean;
   report->live_pairs = (long long)counters[0];
   report->causal_pairs = causal_pairs;
   report->omega_esr = 1.0 - (double)counters[0] / (double)causal_pairs;
   report->live_tiles = (long long)counters[1];
-  report->causal_tiles = (long long)B * H_q * (nq * (nq + 1) / 2);
+  report->causal_tiles = (long long)L * B * H_q * (nq * (nq + 1) / 2);
   report->live_flops = 4.0 * d * kTile * kTile * (double)counters[1];
   if (status & kStatusTimeout) return EA_ERR_TIMEOUT;
   if (status & (kStatusBadLayout | kStatusBadMode)) return EA_ERR_BAD_LAYOUT;
   return EA_OK;
+}
+
+ea_status ea_effective_sparsity(const int32_t* head_mode, const ea_pattern_params* pattern, int B, int S, int H_q,
+                                int H_kv, int d, float* omega_msr_per_sample, ea_sparsity_report* report,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  return stack_sparsity(head_mode, pattern, 1, B, S, H_q, H_kv, d, omega_msr_per_sample, report, workspace,
+                        workspace_bytes, stream);
+}
+
+ea_status ea_model_sparsity(const int32_t* head_mode, const ea_pattern_params* pattern, int L, int B, int S, int H_q,
+                            int H_kv, int d, float* omega_msr_per_sample, ea_sparsity_report* report,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  return stack_sparsity(head_mode, pattern, L, B, S, H_q, H_kv, d, omega_msr_per_sample, report, workspace,
+                        workspace_bytes, stream);
+}
+
+size_t ea_retrieval_workspace_size(int B, int S, int H_q) {
+  if (B < 1 || S < 1 || H_q < 1) return 0;
+  return retrieval_workspace_bytes(B, S, H_q);
+}
+
+ea_status ea_retrieval_scores(const void* q, const void* k, ea_dtype dtype, int B, int S, int H_q, int H_kv, int d,
+                              int needle_begin, int needle_end, float softmax_scale, float* scores, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (!q || !k || !scores) return EA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k)) return EA_ERR_INVALID_ARG;
+  if (B < 1 || S < 1 || H_q < 1 || H_kv < 1 || H_q % H_kv != 0) return EA_ERR_INVALID_ARG;
+  if (needle_begin < 0 || needle_end < needle_begin || needle_end > S) return EA_ERR_INVALID_ARG;
+  if (!(softmax_scale >= 0.f) || std::isinf(softmax_scale)) return EA_ERR_INVALID_ARG;
+  if (dtype != EA_DT_BF16 && dtype != EA_DT_F32) return EA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return EA_ERR_UNSUPPORTED;
+  if ((long long)B * S * H_q * d > (1LL << 40)) return EA_ERR_UNSUPPORTED;
+  if (ea_status s = check_ws(workspace, workspace_bytes, retrieval_workspace_bytes(B, S, H_q))) return s;
+  const double scale = softmax_scale > 0.f ? (double)softmax_scale : 1.0 / std::sqrt((double)d);
+  return launch_retrieval(q, k, dtype, B, S, H_q, H_kv, d, needle_begin, needle_end,
+                          (float)(scale * 1.4426950408889634), scores, workspace, as_stream(stream));
+}
+
+ea_status ea_static_head_assignment(const float* scores, int L, int B, int H_q, int H_kv, double omega_msr,
+                                    int32_t* head_mode, void* stream) {
+  if (!scores || !head_mode) return EA_ERR_INVALID_ARG;
+  if (L < 1 || B < 1 || H_q < 1 || H_kv < 1 || H_q % H_kv != 0) return EA_ERR_INVALID_ARG;
+  if (!(omega_msr >= 0.0 && omega_msr <= 1.0)) return EA_ERR_INVALID_ARG;
+  if (!assignment_shape_ok(L, H_kv)) return EA_ERR_UNSUPPORTED;
+  const int k_full = (int)std::floor((1.0 - omega_msr) * (double)(L * H_kv));
+  return launch_assignment(scores, L, B, H_q, H_kv, k_full, head_mode, as_stream(stream));
 }
 
 size_t ea_xattn_workspace_size(int B, int S, int H_q, int H_kv, int stride) {

@@ -17,8 +17,9 @@ size_t attn_workspace_bytes(int B, int S, int H_q, int H_kv);
 int n_pairs(int H_q, int H_kv);
 ea_status launch_schedule(const int32_t* head_mode, const PatternDev& pat, int B, int S, int H_q, int H_kv,
                           void* workspace, cudaStream_t st);
+// clear: zero the counters first (otherwise the launch adds to them, e.g. layer after layer).
 ea_status launch_sparsity(const int32_t* head_mode, const PatternDev& pat, int B, int S, int H_q, int H_kv,
-                          void* workspace, cudaStream_t st);
+                          void* workspace, cudaStream_t st, bool clear = true);
 // S: query rows of this call (q and o); S_k: rows of k and v.  pat.q_tile0 * 128 is the
 // position of the first query row in the sequence.
 ea_status launch_attn_simt(const float* q, const float* k, const float* v, float* o, const int32_t* head_mode,
@@ -33,4 +34,13 @@ size_t xattn_workspace_bytes(int B, int S, int H_q, int H_kv, int stride);
 ea_status launch_xattn(const void* q, const void* k, const int32_t* head_mode, const PatternDev& pd, int B, int S,
                        int H_q, int H_kv, int stride, float tau, int32_t* row_ptr, int32_t* cols, float* scores,
                        void* workspace, cudaStream_t st);
+
+// Retrieval scores and static assignment (ea_assign.cu).
+size_t retrieval_workspace_bytes(int B, int S, int H_q);
+ea_status launch_retrieval(const void* q, const void* k, ea_dtype dtype, int B, int S, int H_q, int H_kv, int d,
+                           int needle_begin, int needle_end, float scale_log2, float* scores, void* workspace,
+                           cudaStream_t st);
+bool assignment_shape_ok(int L, int H_kv);
+ea_status launch_assignment(const float* scores, int L, int B, int H_q, int H_kv, int k_full, int32_t* head_mode,
+                            cudaStream_t st);
 }  // namespace ea

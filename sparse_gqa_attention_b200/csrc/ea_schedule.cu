@@ -174,10 +174,10 @@ ea_status launch_schedule(const int32_t* head_mode, const PatternDev& pat, int B
 }
 
 ea_status launch_sparsity(const int32_t* head_mode, const PatternDev& pat, int B, int S, int H_q, int H_kv,
-                          void* workspace, cudaStream_t st) {
+                          void* workspace, cudaStream_t st, bool clear) {
   char* ws = static_cast<char*>(workspace);
-  if (cudaMemsetAsync(ws + kWsLivePairs, 0, 16, st) != cudaSuccess) return EA_ERR_CUDA;
-  if (cudaMemsetAsync(ws + kWsHeader, 0, (size_t)B * 4, st) != cudaSuccess) return EA_ERR_CUDA;
+  if (clear && cudaMemsetAsync(ws + kWsLivePairs, 0, 16, st) != cudaSuccess) return EA_ERR_CUDA;
+  if (clear && cudaMemsetAsync(ws + kWsHeader, 0, (size_t)B * 4, st) != cudaSuccess) return EA_ERR_CUDA;
   dim3 grid(pat.n_qt, H_kv, B);
   sparsity_kernel<<<grid, kTile, 0, st>>>(head_mode, pat, S, H_kv, H_q / H_kv,
                                           reinterpret_cast<unsigned long long*>(ws + kWsLivePairs),

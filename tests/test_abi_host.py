@@ -18,7 +18,7 @@ def lib():
 
 def test_every_declared_symbol_is_exported(lib):
     names = abi.declared_symbols()
-    assert len(names) == 14
+    assert len(names) == 18
     for n in names:
         assert hasattr(lib, n), n
 
@@ -136,3 +136,30 @@ def test_xattn_workspace_size(lib):
     assert abi.ea_xattn_workspace_size(B, S, H_q, H_kv, 6) == 0
     assert abi.ea_xattn_workspace_size(B, 1001, H_q, H_kv, 8) == 0
     assert abi.xattn_cols_capacity(2, 300, 3) == 2 * 3 * 3 * 4 // 2
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(n1=300), abi.EA_ERR_INVALID_ARG),            # needle past S
+    (dict(n0=20, n1=10), abi.EA_ERR_INVALID_ARG),
+    (dict(d=96), abi.EA_ERR_UNSUPPORTED),
+    (dict(H_q=7), abi.EA_ERR_INVALID_ARG),
+    (dict(ws=8), abi.EA_ERR_INVALID_ARG),
+    (dict(scale=-1.0), abi.EA_ERR_INVALID_ARG),
+])
+def test_retrieval_argument_checks(lib, case, expect):
+    S, H_q, d = 256, case.get("H_q", 8), case.get("d", 128)
+    st = lib.ea_retrieval_scores(FAKE, FAKE, abi.EA_DT_BF16, 1, S, H_q, 2, d, case.get("n0", 10), case.get("n1", 20),
+                                 case.get("scale", 0.0), FAKE, ctypes.c_void_p(0x100000), case.get("ws", 1 << 30), None)
+    assert st == expect
+
+
+def test_assignment_and_stack_argument_checks(lib):
+    assert lib.ea_static_head_assignment(FAKE, 4, 1, 8, 2, 1.5, FAKE, None) == abi.EA_ERR_INVALID_ARG
+    assert lib.ea_static_head_assignment(FAKE, 4, 1, 8, 3, 0.5, FAKE, None) == abi.EA_ERR_INVALID_ARG
+    assert lib.ea_static_head_assignment(FAKE, 2000, 1, 8, 8, 0.5, FAKE, None) == abi.EA_ERR_UNSUPPORTED
+    assert lib.ea_static_head_assignment(None, 4, 1, 8, 2, 0.5, FAKE, None) == abi.EA_ERR_INVALID_ARG
+    pp, keep = _pattern(2)
+    rep = abi.SparsityReport()
+    assert lib.ea_model_sparsity(FAKE, ctypes.byref(pp), 0, 1, 256, 8, 2, 128, None, ctypes.byref(rep),
+                                 ctypes.c_void_p(0x100000), 1 << 30, None) == abi.EA_ERR_INVALID_ARG
+    assert abi.ea_retrieval_workspace_size(1, 32768, 32) % 256 == 0

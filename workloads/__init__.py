@@ -11,5 +11,5 @@ from .generate import (  # noqa: F401
     WORKLOADS, Workload, Pattern,
     bf16_bits_from_f32, f32_from_bf16_bits,
     attention_inputs, hidden_states, router_weights, block_layout, pattern_for,
-    forced_head_mode, routing_targets, load_router_tuning, positional_component,
+    forced_head_mode, routing_targets, load_router_tuning, positional_component, probe_layer_inputs,
 )

@@ -35,7 +35,7 @@ FULL, STREAMING, BLOCK_SPARSE, STREAMING_BLOCKS = 0, 1, 2, 3
 
 # Stream ids keep the draws of different tensors independent of each other.
 _SID_Q, _SID_K, _SID_V, _SID_HIDDEN, _SID_WK = 11, 12, 13, 14, 15
-_SID_MLP, _SID_ROUTE, _SID_LAYOUT, _SID_SINK = 16, 17, 18, 19
+_SID_MLP, _SID_ROUTE, _SID_LAYOUT, _SID_SINK, _SID_PROBE = 16, 17, 18, 19, 20
 _ROW_CHUNK = 1024
 
 _TUNING_PATH = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
@@ -369,6 +369,29 @@ def pattern_for(w: Workload, layout=None) -> Pattern:
     return Pattern(n_sink=w.n_sink, window=w.window, block=w.block, row_ptr=row_ptr, cols=cols,
                    kind_if_dense=np.asarray(w.kind_if_dense, np.int8),
                    kind_if_sparse=np.asarray(w.kind_if_sparse, np.int8))
+
+
+def probe_layer_inputs(w: Workload, layer: int, needle=(0, 0), amp: float = 6.0):
+    """q, k of one layer of a retrieval probe (appendix C.1 "Retrieval Score Calculation"): the
+    workload's q/k draws for seed (w.seed, layer), plus, for each KV head h, a unit direction u
+    added with amplitude amp to the keys of the needle span and with amplitude amp * a[h] to the
+    last query row of every query head of the group; the per-head affinities a[h] ~ U(0, 1.5) make
+    the heads' needle masses differ.  Storage form like attention_inputs."""
+    import dataclasses as _dc
+    wl_ = _dc.replace(w, seed=w.seed * 1000 + layer + 1)
+    q, k, _ = attention_inputs(wl_)
+    q = f32_from_bf16_bits(q) if q.dtype == np.uint16 else q.copy()
+    k = f32_from_bf16_bits(k) if k.dtype == np.uint16 else k.copy()
+    r = _rng(w.seed, _SID_PROBE, layer)
+    aff = r.uniform(0.0, 1.5, w.H_kv)
+    G = w.H_q // w.H_kv
+    n0, n1 = needle
+    for h in range(w.H_kv):
+        u = r.standard_normal(w.d)
+        u = (u / np.linalg.norm(u)).astype(np.float32)
+        k[:, n0:n1, h, :] += np.float32(amp) * u
+        q[:, w.S - 1, h * G:(h + 1) * G, :] += np.float32(amp * aff[h]) * u
+    return _storage(q, w.dtype), _storage(k, w.dtype)
 
 
 def forced_head_mode(w: Workload, n_sparse: int) -> np.ndarray:
