@@ -67,6 +67,9 @@ class Workload:
     tau: float = 0.9                # XAttention threshold
     pos_amp: float = 0.0            # amplitude of the positional component of q and k
     sink_amp: float = 0.0           # amplitude of the sink direction (all q rows, the first 4 k rows)
+    layers: int = 1                 # > 1: a stack with static retrieval-head assignment
+    needle: tuple = (0, 0)          # retrieval probe needle span [begin, end)
+    omega_static: float = 0.5       # target Omega_MSR of the static assignment
 
     @property
     def G(self) -> int:
@@ -127,6 +130,10 @@ WORKLOADS = {w.name: w for w in [
     _w("llama3-8b-s32k-xassa", 1, 32768, 4096, 32, 8, 128, "bf16", 128, 2048, (STREAMING,) * 8,
        ("fixed", 4), kinds_dense=(BLOCK_SPARSE,) * 8,
        note="XA-SSA: dense heads XAttention (stride 8, tau 0.9), sparse heads streaming", pos_amp=1.7, **_XA),
+    # Static retrieval-head assignment over a stack of layers (probe q/k per layer, shared v).
+    _w("llama3-8b-s32k-stack8", 1, 32768, 4096, 32, 8, 128, "bf16", 128, 2048, (STREAMING,) * 8,
+       ("fixed", 4), layers=8, needle=(16384, 16448), omega_static=0.5,
+       note="8 layers; k = floor(0.5 * 8 * 8) = 32 KV heads keep full attention, 32 stream"),
     _w("small-xattn-g4-s2560", 2, 2560, 256, 8, 2, 128, "bf16", 64, 300, (BLOCK_SPARSE,) * 2,
        ("per_sample", (1, 2)), pos_amp=1.5, **_XA),
     _w("small-xattn-g7-s1000", 1, 1000, 384, 14, 2, 128, "bf16", 0, 1, (BLOCK_SPARSE,) * 2,
