@@ -369,7 +369,7 @@ def run_stack(args):
     pat = abi.Pattern.from_workloads(pat_np)
     scores = torch.empty((L, w.B, w.H_q), dtype=torch.float32, device=dev)
     hm = torch.empty((L, w.B, w.H_kv), dtype=torch.int32, device=dev)
-    rws = torch.zeros(abi.ea_retrieval_workspace_size(w.B, w.S, w.H_q), dtype=torch.uint8, device=dev)
+    rws = torch.zeros(abi.ea_retrieval_workspace_size(w.B, w.S, w.H_q, w.H_kv), dtype=torch.uint8, device=dev)
     aws = torch.zeros(abi.ea_attn_workspace_size(w.B, w.S, w.H_q, w.H_kv), dtype=torch.uint8, device=dev)
     n0, n1 = w.needle
 
@@ -515,7 +515,7 @@ def run_stack(args):
                                "achieved": round(probe_bytes / (probe_max * 1e-3) / 1e9, 1), "peak": pk["hbm"],
                                "unit": "GB/s", "frac": round(probe_bytes / (probe_max * 1e-3) / 1e9 / pk["hbm"], 4),
                                "bytes": probe_bytes, "ms": round(probe_max, 4),
-                               "note": "K re-read once per query head of its group (from L2 after the first)"},
+                               "note": "algorithmic bytes: every layer's K once plus its last q rows"},
             "e2e": {"value": round(whole_job_tflops(live_flops, world, e2e_max), 3), "unit": "TFLOP/s",
                     "ms_per_step": round(e2e_max, 3), "steps": n_e2e, "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h),

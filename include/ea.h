@@ -22,7 +22,8 @@
  *    q, k, v, o and hidden must be 16-byte aligned.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Calls enqueue work on it and return without waiting, except
- *    ea_effective_sparsity and ea_workspace_status, which synchronise it.
+ *    ea_effective_sparsity, ea_model_sparsity and ea_workspace_status, which
+ *    synchronise it.
  *  - Errors: argument checks run on the host before any launch and return
  *    EA_ERR_INVALID_ARG or EA_ERR_UNSUPPORTED with nothing enqueued.  A
  *    failed launch returns EA_ERR_CUDA.  Problems only the device can see (a
@@ -276,11 +277,11 @@ EA_API ea_status ea_model_sparsity(const int32_t* head_mode, const ea_pattern_pa
  * ---------------------------------------------------------------------- */
 
 /* Bytes of workspace ea_retrieval_scores needs (per-slice partial sums). */
-EA_API size_t ea_retrieval_workspace_size(int B, int S, int H_q);
+EA_API size_t ea_retrieval_workspace_size(int B, int S, int H_q, int H_kv);
 
 /* One layer's retrieval scores.  q: device [B, S, H_q, d], k: device
  * [B, S, H_kv, d] (bf16 or f32, 16-byte aligned; only q row S-1 is read);
- * d in {64, 128}; 0 <= needle_begin <= needle_end <= S; softmax_scale 0
+ * d in {64, 128}; H_q / H_kv <= 64; 0 <= needle_begin <= needle_end <= S; softmax_scale 0
  * selects 1/sqrt(d).  scores: device float [B, H_q] (written).  fp32
  * accumulation. */
 EA_API ea_status ea_retrieval_scores(const void* q, const void* k, ea_dtype dtype, int B, int S, int H_q,

@@ -103,7 +103,7 @@ def _lib():
         lib.ea_model_sparsity.argtypes = [c_void_p, POINTER(PatternParams), c_int, c_int, c_int, c_int, c_int, c_int,
                                           c_void_p, POINTER(SparsityReport), c_void_p, c_size_t, c_void_p]
         lib.ea_retrieval_workspace_size.restype = c_size_t
-        lib.ea_retrieval_workspace_size.argtypes = [c_int, c_int, c_int]
+        lib.ea_retrieval_workspace_size.argtypes = [c_int, c_int, c_int, c_int]
         lib.ea_retrieval_scores.restype = st
         lib.ea_retrieval_scores.argtypes = [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
                                             c_int, c_float, c_void_p, c_void_p, c_size_t, c_void_p]
@@ -332,8 +332,8 @@ def ea_model_sparsity(head_mode, pattern: Pattern, L, B, S, H_q, H_kv, d, worksp
     return np.array(per[:], np.float64), {f: getattr(rep, f) for f, _ in SparsityReport._fields_}
 
 
-def ea_retrieval_workspace_size(B: int, S: int, H_q: int) -> int:
-    return int(_lib().ea_retrieval_workspace_size(B, S, H_q))
+def ea_retrieval_workspace_size(B: int, S: int, H_q: int, H_kv: int) -> int:
+    return int(_lib().ea_retrieval_workspace_size(B, S, H_q, H_kv))
 
 
 def ea_retrieval_scores(q, k, needle_begin: int, needle_end: int, scores, workspace, softmax_scale: float = 0.0,

@@ -219,9 +219,9 @@ ea_status ea_model_sparsity(const int32_t* head_mode, const ea_pattern_params* p
                         workspace_bytes, stream);
 }
 
-size_t ea_retrieval_workspace_size(int B, int S, int H_q) {
-  if (B < 1 || S < 1 || H_q < 1) return 0;
-  return retrieval_workspace_bytes(B, S, H_q);
+size_t ea_retrieval_workspace_size(int B, int S, int H_q, int H_kv) {
+  if (B < 1 || S < 1 || H_q < 1 || H_kv < 1 || H_q % H_kv != 0) return 0;
+  return retrieval_workspace_bytes(B, S, H_q, H_kv);
 }
 
 ea_status ea_retrieval_scores(const void* q, const void* k, ea_dtype dtype, int B, int S, int H_q, int H_kv, int d,
@@ -234,8 +234,8 @@ ea_status ea_retrieval_scores(const void* q, const void* k, ea_dtype dtype, int 
   if (!(softmax_scale >= 0.f) || std::isinf(softmax_scale)) return EA_ERR_INVALID_ARG;
   if (dtype != EA_DT_BF16 && dtype != EA_DT_F32) return EA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return EA_ERR_UNSUPPORTED;
-  if ((long long)B * S * H_q * d > (1LL << 40)) return EA_ERR_UNSUPPORTED;
-  if (ea_status s = check_ws(workspace, workspace_bytes, retrieval_workspace_bytes(B, S, H_q))) return s;
+  if (H_q / H_kv > 64 || (long long)B * S * H_q * d > (1LL << 40)) return EA_ERR_UNSUPPORTED;
+  if (ea_status s = check_ws(workspace, workspace_bytes, retrieval_workspace_bytes(B, S, H_q, H_kv))) return s;
   const double scale = softmax_scale > 0.f ? (double)softmax_scale : 1.0 / std::sqrt((double)d);
   return launch_retrieval(q, k, dtype, B, S, H_q, H_kv, d, needle_begin, needle_end,
                           (float)(scale * 1.4426950408889634), scores, workspace, as_stream(stream));

@@ -9,9 +9,10 @@
 // router assigns), a KV head's score being the mean of its G query heads' scores over
 // the probe samples; ties go to the lower flat index l * H_kv + h.
 //
-//   retrieval_partial_kernel  grid (splits, H_q, B): the last query row against a slice
-//                             of the keys, online (max, total mass, needle mass) in log2
-//                             units; K is streamed once per query head in 16-byte loads
+//   retrieval_partial_kernel  grid (splits, H_kv, B): the last query rows of a KV group's G
+//                             heads against a slice of the keys, online (max, total mass,
+//                             needle mass) in log2 units; each key row is read once, in
+//                             16-byte loads
 //   retrieval_finish_kernel   combines the slices: score = needle mass / total mass
 //   assign_kernel             one CTA: KV-head means, rank of every head, head_mode
 #include <cuda_runtime.h>
@@ -39,77 +40,112 @@ __device__ __forceinline__ Triple combine(Triple a, Triple b) {
   return {m, a.l * fa + b.l * fb, a.n * fa + b.n * fb};
 }
 
-__device__ __forceinline__ float dot_row(const float* qs, const float* k, int d) {
-  float acc = 0.f;
-  for (int e = 0; e < d; e += 4) {
-    const float4 x = *reinterpret_cast<const float4*>(k + e);
-    acc = fmaf(qs[e], x.x, acc);
-    acc = fmaf(qs[e + 1], x.y, acc);
-    acc = fmaf(qs[e + 2], x.z, acc);
-    acc = fmaf(qs[e + 3], x.w, acc);
-  }
-  return acc;
-}
-__device__ __forceinline__ float dot_row(const float* qs, const __nv_bfloat16* k, int d) {
-  float acc = 0.f;
-  for (int e = 0; e < d; e += 8) {
-    const uint4 x = *reinterpret_cast<const uint4*>(k + e);
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+// x[g] = qs[g] . krow for the ng (<= NG) heads at qs (rows of d floats); the key row is read once.
+template <int NG>
+__device__ __forceinline__ void dot_rows(const float* qs, const float* krow, int d, int ng, float (&x)[NG]) {
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      acc = fmaf(qs[e + 2 * t], __uint_as_float(w[t] << 16), acc);
-      acc = fmaf(qs[e + 2 * t + 1], __uint_as_float(w[t] & 0xffff0000u), acc);
+  for (int g = 0; g < NG; ++g) x[g] = 0.f;
+  for (int e = 0; e < d; e += 4) {
+    const float4 v = *reinterpret_cast<const float4*>(krow + e);
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+      if (g >= ng) break;
+      const float* qg = qs + g * d + e;
+      x[g] = fmaf(qg[0], v.x, fmaf(qg[1], v.y, fmaf(qg[2], v.z, fmaf(qg[3], v.w, x[g]))));
     }
   }
-  return acc;
+}
+template <int NG>
+__device__ __forceinline__ void dot_rows(const float* qs, const __nv_bfloat16* krow, int d, int ng, float (&x)[NG]) {
+#pragma unroll
+  for (int g = 0; g < NG; ++g) x[g] = 0.f;
+  for (int e = 0; e < d; e += 8) {
+    const uint4 v = *reinterpret_cast<const uint4*>(krow + e);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float kf[8];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      kf[2 * t] = __uint_as_float(w[t] << 16);
+      kf[2 * t + 1] = __uint_as_float(w[t] & 0xffff0000u);
+    }
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+      if (g >= ng) break;
+      const float* qg = qs + g * d + e;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) x[g] = fmaf(qg[t], kf[t], x[g]);
+    }
+  }
 }
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// One CTA per (key slice, KV head, sample) serves all G query heads of the group, so every
+// key row is read once; heads are taken in groups of kHeadChunk (registers per thread).
+constexpr int kHeadChunk = 8;
 
 template <typename T>
 __global__ void __launch_bounds__(kRetThreads)
 retrieval_partial_kernel(const T* __restrict__ q, const T* __restrict__ k, int S, int H_q, int H_kv, int d,
                          int needle_begin, int needle_end, float scale_log2, int splits,
                          float* __restrict__ partial) {
-  __shared__ float qs[128];
-  __shared__ Triple red[kRetThreads / 32];
-  const int sp = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int hk = h / (H_q / H_kv);
-  const T* qrow = q + (((size_t)b * S + (S - 1)) * H_q + h) * d;
-  for (int e = threadIdx.x; e < d; e += kRetThreads) qs[e] = to_f(qrow[e]) * scale_log2;
+  extern __shared__ float qs[];                    // [G][d], scaled to log2 units
+  __shared__ Triple red[kRetThreads / 32][kHeadChunk];
+  const int sp = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  const int G = H_q / H_kv;
+  for (int e = threadIdx.x; e < G * d; e += kRetThreads) {
+    const int g = e / d;
+    qs[e] = to_f(q[(((size_t)b * S + (S - 1)) * H_q + hk * G + g) * d + e % d]) * scale_log2;
+  }
   __syncthreads();
   const int chunk = cdiv(S, splits);
   const int j0 = sp * chunk, j1 = min(S, j0 + chunk);
-  Triple t{-INFINITY, 0.f, 0.f};
-  for (int j = j0 + (int)threadIdx.x; j < j1; j += kRetThreads) {
-    const float x = dot_row(qs, k + (((size_t)b * S + j) * H_kv + hk) * d, d);
-    const float in = (j >= needle_begin && j < needle_end) ? 1.f : 0.f;
-    if (x > t.m) {
-      const float f = exp2f(t.m - x);   // 0 while t.m is -inf
-      t.l = t.l * f + 1.f;
-      t.n = t.n * f + in;
-      t.m = x;
-    } else {
-      const float e = exp2f(x - t.m);
-      t.l += e;
-      t.n += in * e;
-    }
-  }
+  for (int g0 = 0; g0 < G; g0 += kHeadChunk) {
+    const int ng = min(kHeadChunk, G - g0);
+    Triple t[kHeadChunk];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    Triple u{__shfl_xor_sync(0xffffffffu, t.m, o), __shfl_xor_sync(0xffffffffu, t.l, o),
-             __shfl_xor_sync(0xffffffffu, t.n, o)};
-    t = combine(t, u);
-  }
-  if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = t;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    Triple a = red[0];
-    for (int w = 1; w < kRetThreads / 32; ++w) a = combine(a, red[w]);
-    float* out = partial + (((size_t)b * H_q + h) * splits + sp) * 3;
-    out[0] = a.m;
-    out[1] = a.l;
-    out[2] = a.n;
+    for (int g = 0; g < kHeadChunk; ++g) t[g] = Triple{-INFINITY, 0.f, 0.f};
+    for (int j = j0 + (int)threadIdx.x; j < j1; j += kRetThreads) {
+      const T* krow = k + (((size_t)b * S + j) * H_kv + hk) * d;
+      float x[kHeadChunk];
+      dot_rows<kHeadChunk>(qs + (size_t)g0 * d, krow, d, ng, x);
+      const float in = (j >= needle_begin && j < needle_end) ? 1.f : 0.f;
+#pragma unroll
+      for (int g = 0; g < kHeadChunk; ++g) {
+        if (g >= ng) break;
+        if (x[g] > t[g].m) {
+          const float f = exp2f(t[g].m - x[g]);   // 0 while the max is -inf
+          t[g].l = t[g].l * f + 1.f;
+          t[g].n = t[g].n * f + in;
+          t[g].m = x[g];
+        } else {
+          const float e = exp2f(x[g] - t[g].m);
+          t[g].l += e;
+          t[g].n += in * e;
+        }
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < kHeadChunk; ++g) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        Triple u{__shfl_xor_sync(0xffffffffu, t[g].m, o), __shfl_xor_sync(0xffffffffu, t[g].l, o),
+                 __shfl_xor_sync(0xffffffffu, t[g].n, o)};
+        t[g] = combine(t[g], u);
+      }
+      if (threadIdx.x % 32 == 0) red[threadIdx.x / 32][g] = t[g];
+    }
+    __syncthreads();
+    if ((int)threadIdx.x < ng) {
+      const int g = threadIdx.x;
+      Triple a = red[0][g];
+      for (int w = 1; w < kRetThreads / 32; ++w) a = combine(a, red[w][g]);
+      float* out = partial + (((size_t)b * H_q + hk * G + g0 + g) * splits + sp) * 3;
+      out[0] = a.m;
+      out[1] = a.l;
+      out[2] = a.n;
+    }
+    __syncthreads();
   }
 }
 
@@ -151,8 +187,8 @@ assign_kernel(const float* __restrict__ scores, int L, int B, int H_q, int H_kv,
   }
 }
 
-int retrieval_splits(int B, int S, int H_q) {
-  const long long heads = (long long)B * H_q;
+int retrieval_splits(int B, int S, int H_kv) {
+  const long long heads = (long long)B * H_kv;
   long long sp = (4LL * 148 + heads - 1) / heads;
   sp = std::min<long long>(sp, std::max(1, cdiv(S, kRetThreads)));
   return (int)std::max<long long>(1, std::min<long long>(sp, 1024));
@@ -160,22 +196,23 @@ int retrieval_splits(int B, int S, int H_q) {
 
 }  // namespace
 
-size_t retrieval_workspace_bytes(int B, int S, int H_q) {
-  return ((size_t)B * H_q * retrieval_splits(B, S, H_q) * 3 * sizeof(float) + 255) / 256 * 256;
+size_t retrieval_workspace_bytes(int B, int S, int H_q, int H_kv) {
+  return ((size_t)B * H_q * retrieval_splits(B, S, H_kv) * 3 * sizeof(float) + 255) / 256 * 256;
 }
 
 ea_status launch_retrieval(const void* q, const void* k, ea_dtype dtype, int B, int S, int H_q, int H_kv, int d,
                            int needle_begin, int needle_end, float scale_log2, float* scores, void* workspace,
                            cudaStream_t st) {
-  const int splits = retrieval_splits(B, S, H_q);
+  const int splits = retrieval_splits(B, S, H_kv);
   float* partial = static_cast<float*>(workspace);
-  dim3 grid(splits, H_q, B);
+  dim3 grid(splits, H_kv, B);
+  const size_t smem = (size_t)H_q / H_kv * d * sizeof(float);
   if (dtype == EA_DT_BF16)
-    retrieval_partial_kernel<__nv_bfloat16><<<grid, kRetThreads, 0, st>>>(
+    retrieval_partial_kernel<__nv_bfloat16><<<grid, kRetThreads, smem, st>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), S, H_q, H_kv, d, needle_begin,
         needle_end, scale_log2, splits, partial);
   else
-    retrieval_partial_kernel<float><<<grid, kRetThreads, 0, st>>>(
+    retrieval_partial_kernel<float><<<grid, kRetThreads, smem, st>>>(
         static_cast<const float*>(q), static_cast<const float*>(k), S, H_q, H_kv, d, needle_begin, needle_end,
         scale_log2, splits, partial);
   if (cudaGetLastError() != cudaSuccess) return EA_ERR_CUDA;

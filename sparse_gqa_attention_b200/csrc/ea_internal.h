@@ -36,7 +36,7 @@ ea_status launch_xattn(const void* q, const void* k, const int32_t* head_mode, c
                        void* workspace, cudaStream_t st);
 
 // Retrieval scores and static assignment (ea_assign.cu).
-size_t retrieval_workspace_bytes(int B, int S, int H_q);
+size_t retrieval_workspace_bytes(int B, int S, int H_q, int H_kv);
 ea_status launch_retrieval(const void* q, const void* k, ea_dtype dtype, int B, int S, int H_q, int H_kv, int d,
                            int needle_begin, int needle_end, float scale_log2, float* scores, void* workspace,
                            cudaStream_t st);

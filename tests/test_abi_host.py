@@ -162,4 +162,5 @@ def test_assignment_and_stack_argument_checks(lib):
     rep = abi.SparsityReport()
     assert lib.ea_model_sparsity(FAKE, ctypes.byref(pp), 0, 1, 256, 8, 2, 128, None, ctypes.byref(rep),
                                  ctypes.c_void_p(0x100000), 1 << 30, None) == abi.EA_ERR_INVALID_ARG
-    assert abi.ea_retrieval_workspace_size(1, 32768, 32) % 256 == 0
+    assert abi.ea_retrieval_workspace_size(1, 32768, 32, 8) % 256 == 0
+    assert abi.ea_retrieval_workspace_size(1, 32768, 30, 8) == 0

@@ -23,7 +23,7 @@ NEEDLE = (400, 432)
 def gpu_scores(w, q, k, needle):
     dq, dk = _gpu.to_dev(q, w.dtype), _gpu.to_dev(k, w.dtype)
     sc = torch.full((w.B, w.H_q), float("nan"), device="cuda")
-    ws = torch.zeros(abi.ea_retrieval_workspace_size(w.B, w.S, w.H_q), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(abi.ea_retrieval_workspace_size(w.B, w.S, w.H_q, w.H_kv), dtype=torch.uint8, device="cuda")
     abi.ea_retrieval_scores(dq, dk, needle[0], needle[1], sc, ws)
     torch.cuda.synchronize()
     return sc
