@@ -41,10 +41,12 @@ __device__ __forceinline__ Triple combine(Triple a, Triple b) {
 }
 
 // x[g] = qs[g] . krow for the ng (<= NG) heads at qs (rows of d floats); the key row is read once.
-template <int NG>
-__device__ __forceinline__ void dot_rows(const float* qs, const float* krow, int d, int ng, float (&x)[NG]) {
+template <int NG, int D>
+__device__ __forceinline__ void dot_rows(const float* qs, const float* krow, int ng, float (&x)[NG]) {
+  constexpr int d = D;
 #pragma unroll
   for (int g = 0; g < NG; ++g) x[g] = 0.f;
+#pragma unroll
   for (int e = 0; e < d; e += 4) {
     const float4 v = *reinterpret_cast<const float4*>(krow + e);
 #pragma unroll
@@ -55,10 +57,12 @@ __device__ __forceinline__ void dot_rows(const float* qs, const float* krow, int
     }
   }
 }
-template <int NG>
-__device__ __forceinline__ void dot_rows(const float* qs, const __nv_bfloat16* krow, int d, int ng, float (&x)[NG]) {
+template <int NG, int D>
+__device__ __forceinline__ void dot_rows(const float* qs, const __nv_bfloat16* krow, int ng, float (&x)[NG]) {
+  constexpr int d = D;
 #pragma unroll
   for (int g = 0; g < NG; ++g) x[g] = 0.f;
+#pragma unroll
   for (int e = 0; e < d; e += 8) {
     const uint4 v = *reinterpret_cast<const uint4*>(krow + e);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -84,9 +88,9 @@ __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float
 // key row is read once; heads are taken in groups of kHeadChunk (registers per thread).
 constexpr int kHeadChunk = 8;
 
-template <typename T>
+template <typename T, int d>
 __global__ void __launch_bounds__(kRetThreads)
-retrieval_partial_kernel(const T* __restrict__ q, const T* __restrict__ k, int S, int H_q, int H_kv, int d,
+retrieval_partial_kernel(const T* __restrict__ q, const T* __restrict__ k, int S, int H_q, int H_kv,
                          int needle_begin, int needle_end, float scale_log2, int splits,
                          float* __restrict__ partial) {
   extern __shared__ float qs[];                    // [G][d], scaled to log2 units
@@ -108,7 +112,7 @@ retrieval_partial_kernel(const T* __restrict__ q, const T* __restrict__ k, int S
     for (int j = j0 + (int)threadIdx.x; j < j1; j += kRetThreads) {
       const T* krow = k + (((size_t)b * S + j) * H_kv + hk) * d;
       float x[kHeadChunk];
-      dot_rows<kHeadChunk>(qs + (size_t)g0 * d, krow, d, ng, x);
+      dot_rows<kHeadChunk, d>(qs + (size_t)g0 * d, krow, ng, x);
       const float in = (j >= needle_begin && j < needle_end) ? 1.f : 0.f;
 #pragma unroll
       for (int g = 0; g < kHeadChunk; ++g) {
@@ -207,14 +211,22 @@ ea_status launch_retrieval(const void* q, const void* k, ea_dtype dtype, int B, 
   float* partial = static_cast<float*>(workspace);
   dim3 grid(splits, H_kv, B);
   const size_t smem = (size_t)H_q / H_kv * d * sizeof(float);
-  if (dtype == EA_DT_BF16)
-    retrieval_partial_kernel<__nv_bfloat16><<<grid, kRetThreads, smem, st>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), S, H_q, H_kv, d, needle_begin,
-        needle_end, scale_log2, splits, partial);
+  const auto* qb = static_cast<const __nv_bfloat16*>(q);
+  const auto* kb = static_cast<const __nv_bfloat16*>(k);
+  const auto* qf = static_cast<const float*>(q);
+  const auto* kf = static_cast<const float*>(k);
+  if (dtype == EA_DT_BF16 && d == 128)
+    retrieval_partial_kernel<__nv_bfloat16, 128><<<grid, kRetThreads, smem, st>>>(
+        qb, kb, S, H_q, H_kv, needle_begin, needle_end, scale_log2, splits, partial);
+  else if (dtype == EA_DT_BF16)
+    retrieval_partial_kernel<__nv_bfloat16, 64><<<grid, kRetThreads, smem, st>>>(
+        qb, kb, S, H_q, H_kv, needle_begin, needle_end, scale_log2, splits, partial);
+  else if (d == 128)
+    retrieval_partial_kernel<float, 128><<<grid, kRetThreads, smem, st>>>(
+        qf, kf, S, H_q, H_kv, needle_begin, needle_end, scale_log2, splits, partial);
   else
-    retrieval_partial_kernel<float><<<grid, kRetThreads, smem, st>>>(
-        static_cast<const float*>(q), static_cast<const float*>(k), S, H_q, H_kv, d, needle_begin, needle_end,
-        scale_log2, splits, partial);
+    retrieval_partial_kernel<float, 64><<<grid, kRetThreads, smem, st>>>(
+        qf, kf, S, H_q, H_kv, needle_begin, needle_end, scale_log2, splits, partial);
   if (cudaGetLastError() != cudaSuccess) return EA_ERR_CUDA;
   const int n = B * H_q;
   retrieval_finish_kernel<<<cdiv(n, 256), 256, 0, st>>>(partial, n, splits, scores);

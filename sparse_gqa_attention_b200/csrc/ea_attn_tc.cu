@@ -12,29 +12,26 @@
 // a snake order.  A work item is 128 query rows of two query heads of one KV
 // group (two "slots"), so every K/V tile brought into shared memory feeds two
 // 128x128 products.  Warp roles, 384 threads:
-//   warp 0      TMA producer: Q tiles of both slots, then the K and V tiles of each
-//               live key tile into separate rings (3 K stages, released as soon as
-//               both Q K^T products finish; 2 V stages, released after the P V
-//               products), 128-byte swizzle, 2 boxes of 64 columns per 128x128
-//               tile.  No cluster multicast.
-//   warp 1      TMEM owner and MMA issuer (one thread): S_s = Q_s K^T (SS MMA,
-//               M=N=128, K=16 steps) into TMEM, then O_s += P_s V (TS MMA: P
-//               read from TMEM, V from shared memory as an MN-major operand).
+//   warp 0      TMA producer: Q tiles of both slots, then the K and V tiles of the
+//               live key tiles through one 3-slot ring in the order the MMAs use
+//               them (K0, K1, V0, K2, V1, ...), 128-byte swizzle, 2 boxes of 64
+//               columns per 128x128 tile.  No cluster multicast.
+//   warp 1      TMEM owner and MMA issuer (one thread): S_s = Q_s K^T into TMEM
+//               (M=N=128, K=16 steps), O_s += P_s V with P_s and V both read from
+//               shared memory (V as an MN-major operand).  For key tile j it issues
+//               S(j+1) before O += P(j) V(j), so the tensor pipe computes the next
+//               scores while the softmax works on the current ones.
 //   warps 4-7   softmax for slot 0, warps 8-11 for slot 1: one thread per query
-//               row (its TMEM lane).  Reads S from TMEM, applies the element rule
-//               only on boundary tiles, keeps a running max that is raised only
-//               when a new maximum exceeds it by 2^8 (the stale max cancels in
-//               the final division), rescales O in TMEM when it is raised, writes
-//               P as bf16 over the S columns, and finally divides O by the row
-//               sum and stores bf16 rows.
-// TMEM: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512) fp32 columns; P_s
-// aliases the first 64 columns of S_s (bf16 pairs).  Before S_s is overwritten
-// by the next Q K^T product, the MMA thread waits for the P V product that reads
-// P_s: tcgen05 only orders MMAs on the same accumulator, so this keeps the P
-// reads ahead of the S writes by construction.
-// Every mbarrier wait is bounded (kWaitLimitNs); on expiry the CTA raises an
-// abort flag, records kStatusTimeout in the workspace status word, drains its
-// own copies and MMAs, frees TMEM and exits.
+//               row (its TMEM lane).  Loads S from TMEM and releases it at once,
+//               applies the element rule only on boundary tiles, keeps a running
+//               max that is raised only when a new maximum exceeds it by 2^8 (the
+//               stale max cancels in the final division), computes P = exp2(.) in
+//               registers, then - once the previous P V product is done - rescales
+//               O in TMEM when the max was raised and writes P as bf16 into shared
+//               memory (the K-major swizzled layout the MMA reads); finally divides
+//               O by the row sum and stores bf16 rows.
+// TMEM: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512) fp32 columns.  Shared
+// memory: Q0 Q1 | P0 P1 | K/V ring x3 (32 KB each) | barriers.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -51,18 +48,18 @@ namespace {
 using namespace sm100;
 
 constexpr int BM = 128, BN = 128, HD = 128;
-constexpr int NK = 3, NV = 2;                          // K stages, V stages
+constexpr int NKV = 3;                                 // K/V ring slots
 constexpr int kThreads = 384;
 constexpr uint32_t kTileBytes = BM * HD * 2;           // 32 KB per 128x128 bf16 tile
 constexpr uint32_t kBoxBytes = kTileBytes / 2;         // one 64-column box
 constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_K = 2 * kTileBytes;
-constexpr uint32_t OFF_V = OFF_K + NK * kTileBytes;
-constexpr uint32_t OFF_BAR = OFF_V + NV * kTileBytes;
+constexpr uint32_t OFF_P = 2 * kTileBytes;
+constexpr uint32_t OFF_KV = 4 * kTileBytes;
+constexpr uint32_t OFF_BAR = OFF_KV + NKV * kTileBytes;
 enum : int {
-  B_QFULL = 0, B_QEMPTY = 2, B_KFULL = 4, B_KEMPTY = B_KFULL + NK, B_VFULL = B_KEMPTY + NK,
-  B_VEMPTY = B_VFULL + NV, B_SFULL = B_VEMPTY + NV, B_PFULL = B_SFULL + 2, B_PVDONE = B_PFULL + 2,
-  B_OFULL = B_PVDONE + 2, B_FIN = B_OFULL + 2, B_NEVER = B_FIN + 1, N_BAR = B_NEVER + 1
+  B_QFULL = 0, B_QEMPTY = 2, B_KVFULL = 4, B_KVEMPTY = B_KVFULL + NKV, B_SFULL = B_KVEMPTY + NKV,
+  B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2, B_PVDONE = B_PFULL + 2, B_OFULL = B_PVDONE + 2,
+  B_FIN = B_OFULL + 2, B_NEVER = B_FIN + 1, N_BAR = B_NEVER + 1
 };
 constexpr uint32_t OFF_TMEM = OFF_BAR + N_BAR * 8;
 constexpr uint32_t OFF_ABORT = OFF_TMEM + 4;
@@ -160,37 +157,31 @@ __device__ __forceinline__ uint64_t v_desc(uint32_t tile, int kk) {
   return sdesc_sw128(tile + (uint32_t)kk * 2048u, kBoxBytes, 1024u);
 }
 
-// S_s = Q_s K^T for the key tile in stage st.  With kSafeAlias the previous P_s V
-// product (which reads P_s inside the S_s columns) is complete before S_s is written.
-template <bool kSafeAlias>
-__device__ __forceinline__ bool issue_qk(const Ctx& c, uint32_t tmem, uint32_t base, int s, int st, bool& pend,
-                                         int pv_cnt) {
-  if (kSafeAlias && pend) {
-    if (!wait(c, c.bar(B_PVDONE + s), (pv_cnt - 1) & 1)) return false;
-    pend = false;
-  }
+// S_s = Q_s K^T for the key tile at kt, once the softmax has loaded the previous S_s.
+__device__ __forceinline__ bool issue_qk(const Ctx& c, uint32_t tmem, uint32_t base, int s, uint32_t kt,
+                                         int& s_cnt) {
+  if (s_cnt > 0 && !wait(c, c.bar(B_SFREE + s), (s_cnt - 1) & 1)) return false;
   fence_after_sync();
-  const uint32_t qt = base + OFF_Q + s * kTileBytes, kt = base + OFF_K + st * kTileBytes;
+  const uint32_t qt = base + OFF_Q + s * kTileBytes;
 #pragma unroll
   for (int kk = 0; kk < HD / 16; ++kk)
     mma_ss(tmem + col_s(s), qk_desc(qt, kk), qk_desc(kt, kk), IDESC_QK, kk > 0 ? 1u : 0u);
   commit(c.bar(B_SFULL + s));
+  ++s_cnt;
   return true;
 }
 
-// O_s (+)= P_s V for the key tile in stage st, once the softmax has written P_s.
-__device__ __forceinline__ bool issue_pv(const Ctx& c, uint32_t tmem, uint32_t base, int s, int st, bool accumulate,
-                                         bool last, int& p_cnt, int& pv_cnt, bool& pend) {
+// O_s (+)= P_s V for the V tile at vt, once the softmax has written P_s.
+__device__ __forceinline__ bool issue_pv(const Ctx& c, uint32_t tmem, uint32_t base, int s, uint32_t vt,
+                                         bool accumulate, bool last, int& p_cnt) {
   if (!wait(c, c.bar(B_PFULL + s), p_cnt & 1)) return false;
   ++p_cnt;
   fence_after_sync();
-  const uint32_t vt = base + OFF_V + st * kTileBytes;
+  const uint32_t pt = base + OFF_P + s * kTileBytes;
 #pragma unroll
   for (int kk = 0; kk < BN / 16; ++kk)
-    mma_ts(tmem + col_o(s), tmem + col_s(s) + 8u * kk, v_desc(vt, kk), IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
+    mma_ss(tmem + col_o(s), qk_desc(pt, kk), v_desc(vt, kk), IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
   commit(c.bar(B_PVDONE + s));
-  ++pv_cnt;
-  pend = true;
   if (last) {
     commit(c.bar(B_OFULL + s));
     commit(c.bar(B_QEMPTY + s));
@@ -198,13 +189,45 @@ __device__ __forceinline__ bool issue_pv(const Ctx& c, uint32_t tmem, uint32_t b
   return true;
 }
 
+// Share of the exponentials taken on the FMA pipe instead of the MUFU unit: one key
+// pair in EA_POLY_EVERY (0: none).  The two softmax warps of an SM sub-partition share
+// its MUFU unit, which each keeps busy for most of a tile.
+#ifndef EA_POLY_EVERY
+#define EA_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = EA_POLY_EVERY;
+
+// 2^t for a pair of arguments on the FMA/ALU pipes: t = n + f with n the nearest integer
+// (added to and subtracted from 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f from the degree-3
+// polynomial interpolating it at the four Chebyshev nodes of [-1/2, 1/2] (coefficients
+// computed for this kernel; max relative error 1.0e-4); 2^n added into the exponent
+// bits.  Arguments are clamped below at -126 (the result is then 2^-126, not 0).
+__device__ __forceinline__ void ex2_pair_fma(uint64_t t2, float& r0, float& r1) {
+  constexpr float kMagic = 12582912.0f;                  // 1.5 * 2^23, bits 0x4B400000
+  constexpr float c0 = 0.99992454052f, c1 = 0.69313675165f, c2 = 0.24263948202f, c3 = 0.05583828315f;
+  float a0, a1;
+  f2_unpack(t2, a0, a1);
+  const uint64_t t = f2_pack(fmaxf(a0, -126.f), fmaxf(a1, -126.f));
+  const uint64_t j = f2_add(t, f2_pack(kMagic, kMagic));
+  const uint64_t n = f2_add(j, f2_pack(-kMagic, -kMagic));
+  const uint64_t fr = f2_fma(n, f2_pack(-1.f, -1.f), t);
+  uint64_t q = f2_fma(f2_pack(c3, c3), fr, f2_pack(c2, c2));
+  q = f2_fma(q, fr, f2_pack(c1, c1));
+  q = f2_fma(q, fr, f2_pack(c0, c0));
+  float q0, q1, j0, j1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(j, j0, j1);
+  r0 = __uint_as_float(__float_as_uint(q0) + ((__float_as_uint(j0) - 0x4B400000u) << 23));
+  r1 = __uint_as_float(__float_as_uint(q1) + ((__float_as_uint(j1) - 0x4B400000u) << 23));
+}
+
 // One 128-key tile of one query row: running max (raised only past kRescaleLog2),
-// row sum, and P = exp2(scale*log2e*s - max) stored as bf16 pairs over the first 64
-// S columns at p_addr.  kMode 0: every key live; 1: causal rule; 2: streaming rule.
-// Returns the factor O must be multiplied by (1 when the max was not raised).
+// row sum, and P = exp2(scale*log2e*s - max) as bf16 pairs in pk (pk[j] holds keys
+// 2j, 2j+1).  kMode 0: every key live; 1: causal rule; 2: streaming rule.  Returns
+// the factor O must be multiplied by (1 when the max was not raised).
 template <int kMode>
 __device__ __forceinline__ float softmax_tile(const float (&x)[BN], int lim, int sink_lim, int win_lim,
-                                              float scale_log2, float& m_ref, float& l, uint32_t p_addr) {
+                                              float scale_log2, float& m_ref, float& l, uint32_t (&pk)[BN / 2]) {
   auto live = [&](int e) {
     if (kMode == 0) return true;
     if (kMode == 1) return e <= lim;
@@ -232,19 +255,21 @@ __device__ __forceinline__ float softmax_tile(const float (&x)[BN], int lim, int
   const uint64_t scale2 = f2_pack(scale_log2, scale_log2), nsub2 = f2_pack(-sub, -sub);
   uint64_t l2 = f2_pack(0.f, 0.f);
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    uint32_t pk[32];
-#pragma unroll
-    for (int e = 0; e < 64; e += 2) {
-      const int e0 = 64 * half + e;
+  for (int e = 0; e < BN; e += 2) {
+    const uint64_t t2 = f2_fma(f2_pack(x[e], x[e + 1]), scale2, nsub2);
+    float e0, e1;
+    if (kPolyEvery > 0 && (e / 2) % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
+      ex2_pair_fma(t2, e0, e1);
+    } else {
       float t0, t1;
-      f2_unpack(f2_fma(f2_pack(x[e0], x[e0 + 1]), scale2, nsub2), t0, t1);
-      const float p0 = live(e0) ? ex2(t0) : 0.f;
-      const float p1 = live(e0 + 1) ? ex2(t1) : 0.f;
-      l2 = f2_add(l2, f2_pack(p0, p1));
-      pk[e / 2] = pack_bf16x2(p0, p1);
+      f2_unpack(t2, t0, t1);
+      e0 = ex2(t0);
+      e1 = ex2(t1);
     }
-    tmem_st32(p_addr + 32 * half, pk);
+    const float p0 = live(e) ? e0 : 0.f;
+    const float p1 = live(e + 1) ? e1 : 0.f;
+    l2 = f2_add(l2, f2_pack(p0, p1));
+    pk[e / 2] = pack_bf16x2(p0, p1);
   }
   float la, lb;
   f2_unpack(l2, la, lb);
@@ -252,7 +277,22 @@ __device__ __forceinline__ float softmax_tile(const float (&x)[BN], int lim, int
   return f;
 }
 
-template <bool kSafeAlias>
+// Row `row` of P into the K-major, 128-byte-swizzled tile at p_tile: keys 64b..64b+63
+// in box b, 16-byte chunk c of a row at chunk position c ^ (row % 8).
+__device__ __forceinline__ void store_p_row(uint32_t p_tile, int row, const uint32_t (&pk)[BN / 2]) {
+#pragma unroll
+  for (int bx = 0; bx < 2; ++bx) {
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+      const uint32_t addr = p_tile + bx * kBoxBytes + (uint32_t)row * 128u + (uint32_t)((ch ^ (row & 7)) << 4);
+      const int j = 32 * bx + 4 * ch;
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[j]), "r"(pk[j + 1]),
+                   "r"(pk[j + 2]), "r"(pk[j + 3])
+                   : "memory");
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o,
@@ -275,7 +315,7 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     tma_prefetch_map(&tm_k);
     tma_prefetch_map(&tm_v);
     for (int i = 0; i < N_BAR; ++i) {
-      const bool softmax_arrive = (i == B_PFULL || i == B_PFULL + 1);
+      const bool softmax_arrive = (i >= B_SFREE && i < B_SFREE + 2) || (i >= B_PFULL && i < B_PFULL + 2);
       mbar_init(c.bar(i), softmax_arrive ? 128u : 1u);
     }
     *c.abort_flag = 0;
@@ -294,8 +334,19 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int q_use[2] = {0, 0};
-      int k_it = 0, v_it = 0;
+      int kv = 0;
       bool ok = true;
+      // One K or V tile into the next ring slot.
+      auto load_tile = [&](const CUtensorMap* map, int h, int ct, int b) -> bool {
+        const int slot = kv % NKV;
+        if (!wait(c, c.bar(B_KVEMPTY + slot), ((kv / NKV) & 1) ^ 1)) return false;
+        const uint32_t dst = base + OFF_KV + slot * kTileBytes;
+        mbar_expect_tx(c.bar(B_KVFULL + slot), kTileBytes);
+        tma_load_4d(dst, map, c.bar(B_KVFULL + slot), 0, h, ct * BN, b);
+        tma_load_4d(dst + kBoxBytes, map, c.bar(B_KVFULL + slot), 64, h, ct * BN, b);
+        ++kv;
+        return true;
+      };
       for (int it = 0; ok; ++it) {
         const int idx = item_index(it, blockIdx.x, gridDim.x);
         if (idx >= n_items) break;
@@ -313,33 +364,18 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           tma_load_4d(dst + kBoxBytes, &tm_q, c.bar(B_QFULL + s), 64, h_q, I.t * BM, I.b);
           ++q_use[s];
         }
+        // Ring order = MMA order: K0, then per tile jj: K(jj+1), V(jj).
+        auto tile = [&](int jj) { return max(0, live_tile(p, I.kind, I.T, jj, I.sink_end, I.win_lo, I.csr_beg)); };
         for (int jj = 0; jj < I.n && ok; ++jj) {
-          const int ct = max(0, live_tile(p, I.kind, I.T, jj, I.sink_end, I.win_lo, I.csr_beg));
-          const int ks = k_it % NK, vs = v_it % NV;
-          ok = wait(c, c.bar(B_KEMPTY + ks), ((k_it / NK) & 1) ^ 1);
-          if (!ok) break;
-          const uint32_t kdst = base + OFF_K + ks * kTileBytes;
-          mbar_expect_tx(c.bar(B_KFULL + ks), kTileBytes);
-          tma_load_4d(kdst, &tm_k, c.bar(B_KFULL + ks), 0, I.h, ct * BN, I.b);
-          tma_load_4d(kdst + kBoxBytes, &tm_k, c.bar(B_KFULL + ks), 64, I.h, ct * BN, I.b);
-          ++k_it;
-          ok = wait(c, c.bar(B_VEMPTY + vs), ((v_it / NV) & 1) ^ 1);
-          if (!ok) break;
-          const uint32_t vdst = base + OFF_V + vs * kTileBytes;
-          mbar_expect_tx(c.bar(B_VFULL + vs), kTileBytes);
-          tma_load_4d(vdst, &tm_v, c.bar(B_VFULL + vs), 0, I.h, ct * BN, I.b);
-          tma_load_4d(vdst + kBoxBytes, &tm_v, c.bar(B_VFULL + vs), 64, I.h, ct * BN, I.b);
-          ++v_it;
+          if (jj == 0) ok = load_tile(&tm_k, I.h, tile(0), I.b);
+          if (ok && jj + 1 < I.n) ok = load_tile(&tm_k, I.h, tile(jj + 1), I.b);
+          if (ok) ok = load_tile(&tm_v, I.h, tile(jj), I.b);
         }
       }
       // Drain: the last copy armed on every barrier has landed before the CTA exits.
-      for (int st = 0; st < NK; ++st) {
-        const int uses = k_it / NK + (st < k_it % NK ? 1 : 0);
-        if (uses > 0) wait_drain(c, c.bar(B_KFULL + st), (uses - 1) & 1);
-      }
-      for (int st = 0; st < NV; ++st) {
-        const int uses = v_it / NV + (st < v_it % NV ? 1 : 0);
-        if (uses > 0) wait_drain(c, c.bar(B_VFULL + st), (uses - 1) & 1);
+      for (int st = 0; st < NKV; ++st) {
+        const int uses = kv / NKV + (st < kv % NKV ? 1 : 0);
+        if (uses > 0) wait_drain(c, c.bar(B_KVFULL + st), (uses - 1) & 1);
       }
 #pragma unroll
       for (int s = 0; s < 2; ++s)
@@ -348,9 +384,8 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int q_use0 = 0, q_use1 = 0, p_cnt0 = 0, p_cnt1 = 0, pv_cnt0 = 0, pv_cnt1 = 0;
-      bool pend0 = false, pend1 = false;
-      int k_it = 0, v_it = 0;
+      int q_use[2] = {0, 0}, s_cnt[2] = {0, 0}, p_cnt[2] = {0, 0};
+      int kv = 0;
       // Test hook for the timeout path: CTA 0 first waits on a barrier nothing arrives on.
       bool ok = !(inject_stall && blockIdx.x == 0) || wait(c, c.bar(B_NEVER), 0);
       for (int it = 0; ok; ++it) {
@@ -358,39 +393,46 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (idx >= n_items) break;
         const Item I = load_item(items, idx, p, head_mode, H_kv, G);
         if (I.n == 0) continue;
-        ok = wait(c, c.bar(B_QFULL + 0), q_use0 & 1);
-        ++q_use0;
+        ok = wait(c, c.bar(B_QFULL + 0), q_use[0] & 1);
+        ++q_use[0];
         if (I.two) {
-          ok = ok && wait(c, c.bar(B_QFULL + 1), q_use1 & 1);
-          ++q_use1;
+          ok = ok && wait(c, c.bar(B_QFULL + 1), q_use[1] & 1);
+          ++q_use[1];
         }
-        // S of the item's first key tile; its K stage is released once both products finish.
-        ok = ok && wait(c, c.bar(B_KFULL + k_it % NK), (k_it / NK) & 1);
-        if (ok) {
-          ok = issue_qk<kSafeAlias>(c, tmem, base, 0, k_it % NK, pend0, pv_cnt0);
-          if (ok && I.two) ok = issue_qk<kSafeAlias>(c, tmem, base, 1, k_it % NK, pend1, pv_cnt1);
-          commit(c.bar(B_KEMPTY + k_it % NK));
-          ++k_it;
+        // S of the item's first key tile; the ring slot is released once both products finish.
+        {
+          const int slot = kv % NKV;
+          ok = ok && wait(c, c.bar(B_KVFULL + slot), (kv / NKV) & 1);
+          if (ok) {
+            const uint32_t kt = base + OFF_KV + slot * kTileBytes;
+            ok = issue_qk(c, tmem, base, 0, kt, s_cnt[0]);
+            if (ok && I.two) ok = issue_qk(c, tmem, base, 1, kt, s_cnt[1]);
+            if (ok) commit(c.bar(B_KVEMPTY + slot));
+            ++kv;
+          }
         }
         for (int jj = 0; jj < I.n && ok; ++jj) {
-          const int vs = v_it % NV, ks = k_it % NK;
           const bool last = jj + 1 == I.n;
-          ok = wait(c, c.bar(B_VFULL + vs), (v_it / NV) & 1);
-          if (ok) ok = issue_pv(c, tmem, base, 0, vs, jj > 0, last, p_cnt0, pv_cnt0, pend0);
-          if (ok && !last) {
-            ok = wait(c, c.bar(B_KFULL + ks), (k_it / NK) & 1);
-            if (ok) ok = issue_qk<kSafeAlias>(c, tmem, base, 0, ks, pend0, pv_cnt0);
+          if (!last) {   // the next scores first: they run while the softmax works on tile jj
+            const int slot = kv % NKV;
+            ok = wait(c, c.bar(B_KVFULL + slot), (kv / NKV) & 1);
+            if (!ok) break;
+            const uint32_t kt = base + OFF_KV + slot * kTileBytes;
+            ok = issue_qk(c, tmem, base, 0, kt, s_cnt[0]);
+            if (ok && I.two) ok = issue_qk(c, tmem, base, 1, kt, s_cnt[1]);
+            if (!ok) break;
+            commit(c.bar(B_KVEMPTY + slot));
+            ++kv;
           }
-          if (ok && I.two) {
-            ok = issue_pv(c, tmem, base, 1, vs, jj > 0, last, p_cnt1, pv_cnt1, pend1);
-            if (ok && !last) ok = issue_qk<kSafeAlias>(c, tmem, base, 1, ks, pend1, pv_cnt1);
-          }
-          if (!last) {
-            commit(c.bar(B_KEMPTY + ks));   // K tile jj+1: both Q K^T products issued
-            ++k_it;
-          }
-          commit(c.bar(B_VEMPTY + vs));     // V tile jj: both P V products issued
-          ++v_it;
+          const int slot = kv % NKV;
+          ok = wait(c, c.bar(B_KVFULL + slot), (kv / NKV) & 1);
+          if (!ok) break;
+          const uint32_t vt = base + OFF_KV + slot * kTileBytes;
+          ok = issue_pv(c, tmem, base, 0, vt, jj > 0, last, p_cnt[0]);
+          if (ok && I.two) ok = issue_pv(c, tmem, base, 1, vt, jj > 0, last, p_cnt[1]);
+          if (!ok) break;
+          commit(c.bar(B_KVEMPTY + slot));
+          ++kv;
         }
       }
       commit(c.bar(B_FIN));                       // every MMA issued here has completed
@@ -402,7 +444,8 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const int s = (warp - 4) / 4;
     const int row = (warp % 4) * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
-    int s_cnt = 0, o_cnt = 0;
+    const uint32_t p_tile = base + OFF_P + s * kTileBytes;
+    int s_cnt = 0, p_cnt = 0, o_cnt = 0;
     bool ok = true;
     for (int it = 0; ok; ++it) {
       const int idx = item_index(it, blockIdx.x, gridDim.x);
@@ -416,6 +459,7 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       for (int jj = 0; jj < I.n; ++jj) {
         const int ct = live_tile(p, I.kind, I.T, jj, I.sink_end, I.win_lo, I.csr_beg);
         ok = wait(c, c.bar(B_SFULL + s), s_cnt & 1);
+        ok = __all_sync(0xffffffffu, ok);
         ++s_cnt;
         if (!ok) break;
         fence_after_sync();
@@ -428,20 +472,30 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 #pragma unroll
           for (int e = 0; e < BN; ++e) x[e] = __uint_as_float(r[e]);
         }
+        fence_before_sync();
+        mbar_arrive(c.bar(B_SFREE + s));   // S_s may be overwritten by the next Q K^T
         // Key j = 128*ct + e is live iff e <= lim (causal) and, for a streaming head,
         // e < sink_lim or e > win_lim.  Unmasked tiles skip the test.
+        uint32_t pk[BN / 2];
         float f;
         if (ct < 0) {
-          f = softmax_tile<1>(x, -1, 0, 0, p.scale_log2, m_ref, l, lane_addr + col_s(s));
+          f = softmax_tile<1>(x, -1, 0, 0, p.scale_log2, m_ref, l, pk);
         } else if (tile_needs_mask(p, I.kind, I.T, ct)) {
           const int lim = i - ct * BN;
           if (kind_el == EA_STREAMING)
-            f = softmax_tile<2>(x, lim, p.n_sink - ct * BN, lim - p.window, p.scale_log2, m_ref, l,
-                                lane_addr + col_s(s));
+            f = softmax_tile<2>(x, lim, p.n_sink - ct * BN, lim - p.window, p.scale_log2, m_ref, l, pk);
           else
-            f = softmax_tile<1>(x, lim, 0, 0, p.scale_log2, m_ref, l, lane_addr + col_s(s));
+            f = softmax_tile<1>(x, lim, 0, 0, p.scale_log2, m_ref, l, pk);
         } else {
-          f = softmax_tile<0>(x, 0, 0, 0, p.scale_log2, m_ref, l, lane_addr + col_s(s));
+          f = softmax_tile<0>(x, 0, 0, 0, p.scale_log2, m_ref, l, pk);
+        }
+        // The previous P_s V product must be done before P_s is rewritten and before O_s
+        // (which it accumulates into) is rescaled.
+        if (p_cnt > 0) {
+          ok = wait(c, c.bar(B_PVDONE + s), (p_cnt - 1) & 1);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          fence_after_sync();
         }
         const bool raise = f != 1.f;
         if (jj > 0 && __any_sync(0xffffffffu, raise)) {   // O (complete up to tile jj-1) *= f
@@ -454,13 +508,17 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
             tmem_st32(lane_addr + col_o(s) + 32 * q4, r);
           }
+          tmem_st_wait();
         }
-        tmem_st_wait();
+        store_p_row(p_tile, row, pk);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // P visible to the tensor core
         fence_before_sync();
         mbar_arrive(c.bar(B_PFULL + s));
+        ++p_cnt;
       }
       if (!ok) break;
       ok = wait(c, c.bar(B_OFULL + s), o_cnt & 1);
+      ok = __all_sync(0xffffffffu, ok);
       ++o_cnt;
       if (!ok) break;
       fence_after_sync();
@@ -547,7 +605,7 @@ ea_status launch_attn_tc(const void* q, const void* k, const void* v, void* o, c
     return EA_ERR_CUDA;
   const long long n_items = (long long)B * H_kv * pat.n_qt * n_pairs(H_q, H_kv);
   const int grid = (int)std::min<long long>(n_items, sm_count());
-  auto kern = hybrid_attn_tc_kernel<true>;
+  auto kern = hybrid_attn_tc_kernel;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) != cudaSuccess)
     return EA_ERR_CUDA;
   char* ws = static_cast<char*>(workspace);
