@@ -40,6 +40,7 @@ ATTN_SOURCES = ("sparse_gqa_attention_b200/csrc/ea_attn_tc.cu", "sparse_gqa_atte
 ATTN_TRAFFIC = {  # source hash -> {workload: bytes per launch}
     "0296169ffe64f919": {"llama3-8b-s32k-streaming": 588227584 + 242138624},
     "7f7dafa317af8ef7": {"llama3-8b-s32k-streaming": 592338944 + 243713536},
+    "c9ec1a166bddf719": {"llama3-8b-s32k-streaming": 572987648 + 234234880},
 }
 
 def attn_source_hash():
@@ -656,6 +657,15 @@ def e2e_measure(args, w, inp, dev, st, weights, pat, forced, rws, aws, o_dev, xw
     for _ in range(max(1, min(args.warmup, 3))):
         rep = step()
     torch.cuda.synchronize()
+    # The host link's rate on this machine (one pinned q copy alone), to read the number against.
+    qd = torch.empty_like(host["q"], device=dev)
+    link = []
+    for _ in range(3):
+        t_a = time.perf_counter()
+        qd.copy_(host["q"], non_blocking=True)
+        torch.cuda.synchronize()
+        link.append(host["q"].numel() * host["q"].element_size() / (time.perf_counter() - t_a) / 1e9)
+    del qd
     n = max(2, min(args.steps, 5))
     t0 = time.perf_counter()
     for _ in range(n):
@@ -676,7 +686,8 @@ def e2e_measure(args, w, inp, dev, st, weights, pat, forced, rws, aws, o_dev, xw
             "d2h_bytes_per_step": int(o_host.numel() * o_host.element_size() + 4 * w.B + 32),
             "api": api + "; pinned host buffers, H2D / compute / D2H on separate streams",
             "timing": "host clock around synchronised steps (first copy issued to last copy done)",
-            "output_check": "bitwise equal to the device-resident step"}
+            "output_check": "bitwise equal to the device-resident step",
+            "host_to_device_gbs": round(max(link), 1)}
 
 
 def router_bandwidth(w, hidden, weights, dev, st):
