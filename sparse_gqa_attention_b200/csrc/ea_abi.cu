@@ -39,7 +39,8 @@ ea_status check_pattern(const int32_t* head_mode, const ea_pattern_params* p, in
   }
   const bool bsa = any_kind(p, H_kv, EA_BLOCK_SPARSE);
   if (bsa && (!p->bs_row_ptr || !p->bs_col || p->bs_nnz < 0)) return EA_ERR_INVALID_ARG;
-  if ((bsa || any_kind(p, H_kv, EA_STREAMING_BLOCKS)) && p->block != kTile) return EA_ERR_UNSUPPORTED;
+  if ((bsa || any_kind(p, H_kv, EA_STREAMING_BLOCKS)) && p->block != kTile && p->block != 64)
+    return EA_ERR_UNSUPPORTED;
   if ((long long)S > (1LL << 30) || (long long)B * S > (1LL << 31)) return EA_ERR_UNSUPPORTED;
   std::memset(out, 0, sizeof(*out));
   out->n_sink = p->n_sink;
@@ -47,7 +48,7 @@ ea_status check_pattern(const int32_t* head_mode, const ea_pattern_params* p, in
   out->block = p->block;
   out->n_qt = cdiv(S_q, kTile);
   out->q_tile0 = q_offset / kTile;
-  out->n_qb = cdiv(S_k, kTile);
+  out->n_qb = cdiv(S_k, (bsa || any_kind(p, H_kv, EA_STREAMING_BLOCKS)) ? p->block : kTile);
   out->row_ptr = bsa ? p->bs_row_ptr : nullptr;
   out->cols = bsa ? p->bs_col : nullptr;
   out->nnz = bsa ? p->bs_nnz : 0;

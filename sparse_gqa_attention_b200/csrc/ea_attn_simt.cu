@@ -24,14 +24,14 @@ __device__ __forceinline__ bool simt_tile_live(const PatternDev& p, int kind, in
     if (c0 < p.n_sink) return true;
     return r0 - (c0 + kKeys - 1) < p.window;  // smallest distance i - j over the tile pair
   }
-  if (kind == EA_STREAMING_BLOCKS)   // block == 128: the 64-row tile sits in one query block
-    return c0 / kTile < cdiv(p.n_sink, kTile) || r0 / kTile - c0 / kTile < cdiv(p.window, kTile);
-  if (kind == EA_BLOCK_SPARSE) {   // block == 128: 64-row and 64-key tiles sit in one block each
-    // (r0 is a sequence position; chunks start on a multiple of 128)
+  const int B = p.block;   // 64 or 128: the 64-row and 64-key tiles sit in one block each
+  if (kind == EA_STREAMING_BLOCKS)
+    return c0 / B < cdiv(p.n_sink, B) || r0 / B - c0 / B < cdiv(p.window, B);
+  if (kind == EA_BLOCK_SPARSE) {   // (r0 is a sequence position; chunks start on a multiple of 128)
     long long a, e;
-    csr_row(p, H_kv, b, h, r0 / kTile, a, e);
+    csr_row(p, H_kv, b, h, r0 / B, a, e);
     for (long long x = a; x < e; ++x)
-      if (p.cols[x] == c0 / kTile) return true;
+      if (p.cols[x] == c0 / B) return true;
     return false;
   }
   return true;

@@ -135,6 +135,8 @@ __device__ __forceinline__ Item load_item(const int4* items, int idx, const Patt
   if (is_streaming(I.kind)) {
     stream_ranges(p, I.kind, I.T, I.sink_end, I.win_lo);
     I.n = I.sink_end + max(0, I.T - I.win_lo + 1);
+  } else if (bs64_kind(p, I.kind)) {
+    I.n = n_live_tiles(p, I.kind, H_kv, I.b, I.h, I.T);
   } else if (I.kind == EA_BLOCK_SPARSE) {
     long long a, e;
     csr_row(p, H_kv, I.b, I.h, I.T, a, e);
@@ -144,6 +146,32 @@ __device__ __forceinline__ Item load_item(const int4* items, int idx, const Patt
     I.n = I.T + 1;
   }
   return I;
+}
+
+// Sequential walk over an item's live key tiles: the tile index (-1: nothing live) and,
+// for block-64 block-sparse heads, the 2x2 map of its live blocks (0xF otherwise).
+struct Walk {
+  Bs64 w;
+  int jj;
+  __device__ __forceinline__ int next(const PatternDev& p, const Item& I, uint32_t& map) {
+    map = 0xFu;
+    int c;
+    if (bs64_kind(p, I.kind)) {
+      c = bs64_next(p, w, map);
+      if (c > I.T) c = -1;   // a block above the diagonal (malformed layout): skipped
+    } else {
+      c = live_tile(p, I.kind, I.T, jj, I.sink_end, I.win_lo, I.csr_beg);
+    }
+    ++jj;
+    return c;
+  }
+};
+__device__ __forceinline__ Walk start_walk(const PatternDev& p, const Item& I, int H_kv) {
+  Walk k;
+  k.jj = 0;
+  k.w.a0 = k.w.e0 = k.w.a1 = k.w.e1 = 0;
+  if (bs64_kind(p, I.kind)) bs64_rows(p, H_kv, I.b, I.h, I.T, k.w);
+  return k;
 }
 
 __device__ __forceinline__ uint64_t qk_desc(uint32_t tile, int kk) {
@@ -223,7 +251,8 @@ __device__ __forceinline__ void ex2_pair_fma(uint64_t t2, float& r0, float& r1) 
 
 // One 128-key tile of one query row: running max (raised only past kRescaleLog2),
 // row sum, and P = exp2(scale*log2e*s - max) as bf16 pairs in pk (pk[j] holds keys
-// 2j, 2j+1).  kMode 0: every key live; 1: causal rule; 2: streaming rule.  Returns
+// 2j, 2j+1).  kMode 0: every key live; 1: causal rule; 2: streaming rule; 3: causal
+// rule within the enabled 64-key halves (block-64 kinds; sink_lim holds the bits).  Returns
 // the factor O must be multiplied by (1 when the max was not raised).
 template <int kMode>
 __device__ __forceinline__ float softmax_tile(const float (&x)[BN], int lim, int sink_lim, int win_lim,
@@ -231,6 +260,7 @@ __device__ __forceinline__ float softmax_tile(const float (&x)[BN], int lim, int
   auto live = [&](int e) {
     if (kMode == 0) return true;
     if (kMode == 1) return e <= lim;
+    if (kMode == 3) return e <= lim && ((sink_lim >> (e >> 6)) & 1) != 0;   // sink_lim: key-half bits
     return e <= lim && (e < sink_lim || e > win_lim);
   };
   auto xm = [&](int e) { return live(e) ? x[e] : -INFINITY; };
@@ -364,12 +394,14 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           tma_load_4d(dst + kBoxBytes, &tm_q, c.bar(B_QFULL + s), 64, h_q, I.t * BM, I.b);
           ++q_use[s];
         }
-        // Ring order = MMA order: K0, then per tile jj: K(jj+1), V(jj).
-        auto tile = [&](int jj) { return max(0, live_tile(p, I.kind, I.T, jj, I.sink_end, I.win_lo, I.csr_beg)); };
+        // Ring order = MMA order: K0, then per tile jj: K(jj+1), V(jj).  The K walk runs
+        // one tile ahead of the V walk.
+        Walk kw = start_walk(p, I, H_kv), vw = start_walk(p, I, H_kv);
+        uint32_t map;
         for (int jj = 0; jj < I.n && ok; ++jj) {
-          if (jj == 0) ok = load_tile(&tm_k, I.h, tile(0), I.b);
-          if (ok && jj + 1 < I.n) ok = load_tile(&tm_k, I.h, tile(jj + 1), I.b);
-          if (ok) ok = load_tile(&tm_v, I.h, tile(jj), I.b);
+          if (jj == 0) ok = load_tile(&tm_k, I.h, max(0, kw.next(p, I, map)), I.b);
+          if (ok && jj + 1 < I.n) ok = load_tile(&tm_k, I.h, max(0, kw.next(p, I, map)), I.b);
+          if (ok) ok = load_tile(&tm_v, I.h, max(0, vw.next(p, I, map)), I.b);
         }
       }
       // Drain: the last copy armed on every barrier has landed before the CTA exits.
@@ -456,8 +488,11 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       const int i_out = I.t * BM + row;    // row of q and o in this call
       const int kind_el = I.kind == EA_STREAMING ? EA_STREAMING : EA_FULL;
       float m_ref = -INFINITY, l = 0.f;
+      const bool blk64 = p.block == 64 && (I.kind == EA_BLOCK_SPARSE || I.kind == EA_STREAMING_BLOCKS);
+      Walk walk = start_walk(p, I, H_kv);
       for (int jj = 0; jj < I.n; ++jj) {
-        const int ct = live_tile(p, I.kind, I.T, jj, I.sink_end, I.win_lo, I.csr_beg);
+        uint32_t map;
+        const int ct = walk.next(p, I, map);
         ok = wait(c, c.bar(B_SFULL + s), s_cnt & 1);
         ok = __all_sync(0xffffffffu, ok);
         ++s_cnt;
@@ -480,6 +515,12 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         float f;
         if (ct < 0) {
           f = softmax_tile<1>(x, -1, 0, 0, p.scale_log2, m_ref, l, pk);
+        } else if (blk64) {   // 64x64 blocks: the key halves this warp's query half may read
+          const int hb = (int)half_bits(p, I.kind, I.T, ct, row >> 6, map);
+          if (hb == 3 && ct < I.T)
+            f = softmax_tile<0>(x, 0, 0, 0, p.scale_log2, m_ref, l, pk);
+          else
+            f = softmax_tile<3>(x, i - ct * BN, hb, 0, p.scale_log2, m_ref, l, pk);
         } else if (tile_needs_mask(p, I.kind, I.T, ct)) {
           const int lim = i - ct * BN;
           if (kind_el == EA_STREAMING)

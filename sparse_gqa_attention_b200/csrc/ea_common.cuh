@@ -11,11 +11,16 @@
 //   STREAMING     sink tiles 0..ceil(n_sink/128)-1 (at most t), then window tiles
 //                 floor(max(0, 128t - window + 1)/128)..t (not repeating sink tiles).
 //                 Every enumerated tile holds at least one live pair.
-//   BLOCK_SPARSE  (block == 128) the listed key blocks of CSR row
-//                 (b*H_kv + h)*n_qt + t; the diagonal tile needs the causal mask.
-//   STREAMING_BLOCKS (block == 128) sink tiles 0..ceil(n_sink/128)-1 (at most t),
-//                 then tiles max(0, t - ceil(window/128) + 1)..t; only the diagonal
-//                 tile needs the causal mask.
+//   BLOCK_SPARSE  block 128: the listed key blocks of CSR row (b*H_kv + h)*n_qb + t;
+//                 the diagonal tile needs the causal mask.  Block 64: the union of
+//                 the key tiles of CSR rows 2t and 2t+1 (key block kb lies in tile
+//                 kb/2), each with a 2x2 map of its live 64x64 blocks.
+//   STREAMING_BLOCKS sink blocks kb < sb = ceil(n_sink/block) and local blocks
+//                 qb - kb < lb = ceil(window/block): sink tiles up to
+//                 ceil(sb*block/128)-1 (at most t), then tiles from
+//                 floor(max(0, q0 - lb + 1)*block/128) to t, q0 = 128t/block the
+//                 tile's first query block.  Block 128: only the diagonal tile needs
+//                 the causal mask; block 64: boundary tiles use the 2x2 block map.
 #pragma once
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -44,7 +49,7 @@ struct PatternDev {
   int block;
   int n_qt;                 // query tiles of this call: ceil(S_q / 128)
   int q_tile0;              // global index of the call's first query tile (q_offset / 128)
-  int n_qb;                 // CSR rows per (b, h_kv): ceil(S_k / 128)
+  int n_qb;                 // CSR rows per (b, h_kv): ceil(S_k / block)
   const int32_t* row_ptr;
   const int32_t* cols;
   long long nnz;
@@ -65,10 +70,15 @@ __device__ __forceinline__ bool is_streaming(int kind) { return kind == EA_STREA
 
 // Tile ranges of query tile t for the two streaming kinds: [0, sink_end) and [win_lo, t].
 __device__ __forceinline__ void stream_ranges(const PatternDev& p, int kind, int t, int& sink_end, int& win_lo) {
-  sink_end = min(cdiv(p.n_sink, kTile), t + 1);
-  const int lo = kind == EA_STREAMING_BLOCKS ? max(0, t - cdiv(p.window, kTile) + 1)
-                                             : max(0, t * kTile - p.window + 1) / kTile;
-  win_lo = max(lo, sink_end);
+  if (kind == EA_STREAMING_BLOCKS) {
+    const int B = p.block, sb = cdiv(p.n_sink, B), lb = cdiv(p.window, B);
+    sink_end = min(cdiv(sb * B, kTile), t + 1);
+    const int q0 = t * (kTile / B);                       // the tile's first query block
+    win_lo = max(max(0, q0 - lb + 1) * B / kTile, sink_end);
+  } else {
+    sink_end = min(cdiv(p.n_sink, kTile), t + 1);
+    win_lo = max(max(0, t * kTile - p.window + 1) / kTile, sink_end);
+  }
 }
 
 // CSR row [beg, end) of (b, h, global query tile t), clamped so a malformed row never
@@ -83,6 +93,44 @@ __device__ __forceinline__ void csr_row(const PatternDev& p, int H_kv, int b, in
   end = e;
 }
 
+// Block-sparse rows of a 128-row query tile at block 64: CSR rows 2t and 2t+1.
+struct Bs64 {
+  long long a0, e0, a1, e1;
+};
+__device__ __forceinline__ void bs64_rows(const PatternDev& p, int H_kv, int b, int h, int t, Bs64& w) {
+  csr_row(p, H_kv, b, h, 2 * t, w.a0, w.e0);
+  if (2 * t + 1 < p.n_qb) {
+    csr_row(p, H_kv, b, h, 2 * t + 1, w.a1, w.e1);
+  } else {
+    w.a1 = w.e1 = 0;
+  }
+}
+// Next key tile of the union of the two rows (ascending), with its 2x2 map: bit
+// 2*qsub + ksub for query half qsub (row 2t+qsub) and key half ksub (block 2c+ksub).
+// Returns -1 when both rows are done.  Every walker over the same rows visits the
+// same sequence, so producer, MMA issuer, softmax and schedule stay in step.
+__device__ __forceinline__ int bs64_next(const PatternDev& p, Bs64& w, uint32_t& map) {
+  const int k0 = w.a0 < w.e0 ? p.cols[w.a0] : 0x7fffffff;
+  const int k1 = w.a1 < w.e1 ? p.cols[w.a1] : 0x7fffffff;
+  const int kmin = min(k0, k1);
+  if (kmin == 0x7fffffff) return -1;
+  const int c = kmin >> 1;
+  map = 0;
+  while (w.a0 < w.e0 && (p.cols[w.a0] >> 1) == c) {
+    map |= 1u << (p.cols[w.a0] & 1);
+    ++w.a0;
+  }
+  while (w.a1 < w.e1 && (p.cols[w.a1] >> 1) == c) {
+    map |= 4u << (p.cols[w.a1] & 1);
+    ++w.a1;
+  }
+  return c;
+}
+
+__device__ __forceinline__ bool bs64_kind(const PatternDev& p, int kind) {
+  return kind == EA_BLOCK_SPARSE && p.block == 64;
+}
+
 // Number of live key tiles of query tile t.
 __device__ __forceinline__ int n_live_tiles(const PatternDev& p, int kind, int H_kv, int b, int h, int t) {
   if (is_streaming(kind)) {
@@ -90,12 +138,34 @@ __device__ __forceinline__ int n_live_tiles(const PatternDev& p, int kind, int H
     stream_ranges(p, kind, t, se, wl);
     return se + max(0, t - wl + 1);
   }
+  if (bs64_kind(p, kind)) {
+    Bs64 w;
+    bs64_rows(p, H_kv, b, h, t, w);
+    uint32_t map;
+    int n = 0;
+    while (bs64_next(p, w, map) >= 0) ++n;
+    return n;
+  }
   if (kind == EA_BLOCK_SPARSE) {
     long long a, e;
     csr_row(p, H_kv, b, h, t, a, e);
     return (int)(e - a);
   }
   return t + 1;
+}
+
+// For block-64 kinds: the enabled key halves (bit ksub) of key tile c for the query
+// half qsub of tile t, from the 2x2 map (block-sparse) or the streaming-block rule.
+__device__ __forceinline__ uint32_t half_bits(const PatternDev& p, int kind, int t, int c, int qsub, uint32_t map) {
+  if (kind == EA_BLOCK_SPARSE) return (map >> (2 * qsub)) & 3u;
+  const int sb = cdiv(p.n_sink, 64), lb = cdiv(p.window, 64), q = 2 * t + qsub;
+  uint32_t bits = 0;
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+    const int kb = 2 * c + ks;
+    if (kb <= q && (kb < sb || q - kb < lb)) bits |= 1u << ks;
+  }
+  return bits;
 }
 
 // Key tile index of the jj-th live tile (0 <= jj < n_live_tiles).  For block-sparse
@@ -124,8 +194,8 @@ __device__ __forceinline__ bool key_live(const PatternDev& p, int kind, int i, i
   if (j > i) return false;
   if (kind == EA_STREAMING) return j < p.n_sink || i - j < p.window;
   if (kind == EA_STREAMING_BLOCKS)
-    return j / kTile < cdiv(p.n_sink, kTile) || i / kTile - j / kTile < cdiv(p.window, kTile);
-  return true;  // FULL, and BLOCK_SPARSE inside a listed tile (block == tile)
+    return j / p.block < cdiv(p.n_sink, p.block) || i / p.block - j / p.block < cdiv(p.window, p.block);
+  return true;  // FULL, and BLOCK_SPARSE inside a listed block
 }
 
 }  // namespace ea

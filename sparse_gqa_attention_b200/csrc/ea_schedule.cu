@@ -56,19 +56,24 @@ schedule_kernel(const int32_t* __restrict__ head_mode, PatternDev p, int H_kv, i
     const int m = head_mode[b * H_kv + h];
     if (m != 0 && m != 1) bad |= kStatusBadMode;
     const int kind = head_kind(p, head_mode, H_kv, b, h);
-    if (kind == EA_BLOCK_SPARSE && pr == 0) {
-      const long long r = ((long long)b * H_kv + h) * p.n_qb + t;
-      const long long a0 = p.row_ptr[r], a1 = p.row_ptr[r + 1];
-      if (a0 < 0 || a1 < a0 || a1 > p.nnz || a1 == a0) {
-        bad |= kStatusBadLayout;
-      } else {
-        int prev = -1;
-        for (long long e = a0; e < a1; ++e) {
-          const int c = p.cols[e];
-          if (c <= prev || c > t) bad |= kStatusBadLayout;
-          prev = c;
+    if (kind == EA_BLOCK_SPARSE && pr == 0) {   // the tile's CSR rows (1 at block 128, 2 at 64)
+      const int per = kTile / p.block;
+      for (int u = 0; u < per; ++u) {
+        const int qb = t * per + u;
+        if (qb >= p.n_qb) break;
+        const long long r = ((long long)b * H_kv + h) * p.n_qb + qb;
+        const long long a0 = p.row_ptr[r], a1 = p.row_ptr[r + 1];
+        if (a0 < 0 || a1 < a0 || a1 > p.nnz || a1 == a0) {
+          bad |= kStatusBadLayout;
+        } else {
+          int prev = -1;
+          for (long long e = a0; e < a1; ++e) {
+            const int c = p.cols[e];
+            if (c <= prev || c > qb) bad |= kStatusBadLayout;
+            prev = c;
+          }
+          if (prev != qb) bad |= kStatusBadLayout;
         }
-        if (prev != t) bad |= kStatusBadLayout;
       }
     }
     atomicAdd(&bins[item_cost(p, head_mode, H_kv, G, b, h, t, pr, n_bins)], 1);
@@ -118,19 +123,21 @@ sparsity_kernel(const int32_t* __restrict__ head_mode, PatternDev p, int S, int 
     if (kind == EA_STREAMING) {
       cnt = min(i + 1, p.window) + max(0, min(p.n_sink, i - p.window + 1));
     } else if (kind == EA_STREAMING_BLOCKS) {
-      const long long local_start = (long long)max(0, t - cdiv(p.window, kTile) + 1) * kTile;
-      cnt = (i - local_start + 1) + max(0LL, min((long long)cdiv(p.n_sink, kTile) * kTile, local_start));
+      const int B = p.block, qb = i / B;
+      const long long local_start = (long long)max(0, qb - cdiv(p.window, B) + 1) * B;
+      cnt = (i - local_start + 1) + max(0LL, min((long long)cdiv(p.n_sink, B) * B, local_start));
     } else if (kind == EA_BLOCK_SPARSE) {
+      const int B = p.block, qb = i / B;
       long long a, e;
-      csr_row(p, H_kv, b, h, t, a, e);
+      csr_row(p, H_kv, b, h, qb, a, e);
       int below = 0;
       bool diag = false;
       for (long long x = a; x < e; ++x) {
         const int c = p.cols[x];
-        below += (c >= 0 && c < t);
-        diag |= (c == t);
+        below += (c >= 0 && c < qb);
+        diag |= (c == qb);
       }
-      cnt = (long long)below * kTile + (diag ? (i - t * kTile + 1) : 0);
+      cnt = (long long)below * B + (diag ? (i - qb * B + 1) : 0);
     } else {
       cnt = i + 1;
     }

@@ -41,6 +41,7 @@ def _chunked(w, q, k, v, mode, pat, chunk):
 
 
 @pytest.mark.parametrize("name,chunk", [("small-mixed-g4-s1000", 256), ("small-blockstream-g4-s900", 384),
+                                        ("small-b64-g4-s1000", 256), ("small-fp32-b64-s700", 128),
                                         ("small-bsa-g7-s777", 128), ("small-fp32-d128-s300", 128),
                                         ("tiny-fp32-s512", 256)])
 def test_chunks_equal_one_call(name, chunk):

@@ -20,9 +20,11 @@ from tests import _gpu
 pytestmark = pytest.mark.gpu
 
 SMALL = ["tiny-fp32-s512", "small-mixed-g4-s1000", "small-bsa-g7-s777", "small-stream-g1-s700",
-         "small-fp32-d128-s300", "small-blockstream-g4-s900", "small-fp32-blockstream-s400"]
+         "small-fp32-d128-s300", "small-blockstream-g4-s900", "small-fp32-blockstream-s400",
+         "small-b64-g4-s1000", "small-b64-g7-s777", "small-fp32-b64-s700"]
 FULL = ["llama3-8b-s32k-streaming", "qwen-g7-s64k-blocksparse", "llama3-8b-b4-s16k-mixed",
-        "llama3-8b-s128k-sweep", "llama3-8b-s32k-blockstream"]
+        "llama3-8b-s128k-sweep", "llama3-8b-s32k-blockstream", "qwen-g7-s64k-blocksparse-b64",
+        "llama3-8b-s32k-blockstream-b64"]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -107,6 +109,35 @@ def test_attention_edge_shapes(S, H_q, H_kv, n_sink, window, kinds, dtype):
     q, k, v = wl.attention_inputs(w)
     pat = wl.pattern_for(w)
     mode = np.array([[1] * H_kv, [h % 2 for h in range(H_kv)]], np.int32)
+    got, status = _gpu.run_attention(w, q, k, v, mode, pat)
+    assert status == abi.EA_OK
+    _gpu.assert_close(got, _gpu.oracle_attention(w, q, k, v, mode, pat), dtype, w.name)
+
+
+EDGE64 = [  # block 64: (S, n_sink, window, sparse kinds, dtype)
+    (1, 0, 1, (2, 3), "bf16"),
+    (63, 1, 1, (2, 3), "bf16"),
+    (64, 64, 64, (3, 2), "bf16"),
+    (65, 0, 65, (2, 3), "bf16"),
+    (127, 130, 1, (3, 2), "bf16"),
+    (129, 0, 1, (2, 2), "bf16"),
+    (300, 64, 128, (3, 3), "bf16"),
+    (383, 200, 1000, (2, 3), "bf16"),
+    (65, 1, 64, (2, 3), "f32"),
+    (300, 65, 129, (3, 2), "f32"),
+]
+
+
+@pytest.mark.parametrize("S,n_sink,window,kinds,dtype", EDGE64)
+def test_attention_block64_edges(S, n_sink, window, kinds, dtype):
+    """The pages' block edge 64 (appendix D.1): every 128x128 tile holds 2x2 blocks, so
+    ragged block rows, half-live tiles and the diagonal block halves are all exercised."""
+    base = wl.WORKLOADS["small-b64-g4-s1000"]
+    w = dataclasses.replace(base, name=f"edge64-{S}", B=2, S=S, n_sink=n_sink, window=window,
+                            kind_if_dense=(0, 0), kind_if_sparse=tuple(kinds), dtype=dtype, density=0.4)
+    q, k, v = wl.attention_inputs(w)
+    pat = wl.pattern_for(w)
+    mode = np.array([[1, 1], [0, 1]], np.int32)
     got, status = _gpu.run_attention(w, q, k, v, mode, pat)
     assert status == abi.EA_OK
     _gpu.assert_close(got, _gpu.oracle_attention(w, q, k, v, mode, pat), dtype, w.name)

@@ -130,6 +130,18 @@ WORKLOADS = {w.name: w for w in [
     _w("llama3-8b-s32k-xassa", 1, 32768, 4096, 32, 8, 128, "bf16", 128, 2048, (STREAMING,) * 8,
        ("fixed", 4), kinds_dense=(BLOCK_SPARSE,) * 8,
        note="XA-SSA: dense heads XAttention (stride 8, tau 0.9), sparse heads streaming", pos_amp=1.7, **_XA),
+    # The pages' block edge, 64 (appendix D.1): block-sparse and block-granular streaming heads.
+    _w("small-b64-g4-s1000", 2, 1000, 256, 8, 2, 128, "bf16", 128, 300, (STREAMING_BLOCKS, BLOCK_SPARSE),
+       ("per_sample", (1, 2)), block=64, density=0.3),
+    _w("small-b64-g7-s777", 1, 777, 384, 14, 2, 128, "bf16", 0, 1, (BLOCK_SPARSE,) * 2, ("fixed", 1),
+       block=64, density=0.3),
+    _w("small-fp32-b64-s700", 2, 700, 256, 4, 2, 64, "f32", 100, 129, (BLOCK_SPARSE, STREAMING_BLOCKS),
+       ("per_sample", (1, 2)), block=64, density=0.4),
+    _w("qwen-g7-s64k-blocksparse-b64", 1, 65536, 3584, 28, 4, 128, "bf16", 128, 2048, (BLOCK_SPARSE,) * 4,
+       ("fixed", 2), block=64, note="config 3 at the pages' block edge 64: first + diagonal + 10% of causal blocks"),
+    _w("llama3-8b-s32k-blockstream-b64", 1, 32768, 4096, 32, 8, 128, "bf16", 128, 2048,
+       (STREAMING_BLOCKS,) * 8, ("fixed", 4), block=64,
+       note="the Llama layer with streaming heads at 64-key blocks (2 sink blocks, 32 local blocks)"),
     # Static retrieval-head assignment over a stack of layers (probe q/k per layer, shared v).
     _w("llama3-8b-s32k-stack8", 1, 32768, 4096, 32, 8, 128, "bf16", 128, 2048, (STREAMING,) * 8,
        ("fixed", 4), layers=8, needle=(16384, 16448), omega_static=0.5,
