@@ -328,7 +328,8 @@ def run_cuda(args):
             "router_roofline": router_full,
             **({"xattn_roofline": xattn_line} if xattn_line else {}),
             "e2e": e2e,
-            "gpu_launches": (11 if xattn else 6) * args.steps,
+            # router 3 + (XAttention 5) + schedule 2 + attention 1 + sparsity 1 per step
+            "gpu_launches": (12 if xattn else 7) * args.steps,
             "clocks": clk.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -529,7 +530,7 @@ def run_stack(args):
                     "api": "per layer ea_build_schedule + ea_attn_scheduled, then ea_model_sparsity; pinned host "
                            "buffers, layer l+1's q/k copied while layer l runs",
                     "timing": "host clock around synchronised steps"},
-            "gpu_launches": 2 * L * args.steps + args.steps,
+            "gpu_launches": 4 * L * args.steps,     # per layer: schedule 2 + attention 1 + its sparsity count 1
             "clocks": clk.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

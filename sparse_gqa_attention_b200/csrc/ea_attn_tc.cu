@@ -149,7 +149,9 @@ __device__ __forceinline__ Item load_item(const int4* items, int idx, const Patt
 }
 
 // Sequential walk over an item's live key tiles: the tile index (-1: nothing live) and,
-// for block-64 block-sparse heads, the 2x2 map of its live blocks (0xF otherwise).
+// for block-64 block-sparse heads, the 2x2 map of its live blocks (0xF otherwise).  The
+// block-64 state exists only in the kernel instance launched for block-64 patterns.
+template <bool kB64>
 struct Walk {
   Bs64 w;
   int jj;
@@ -166,11 +168,22 @@ struct Walk {
     return c;
   }
 };
-__device__ __forceinline__ Walk start_walk(const PatternDev& p, const Item& I, int H_kv) {
-  Walk k;
+template <>
+struct Walk<false> {
+  int jj;
+  __device__ __forceinline__ int next(const PatternDev& p, const Item& I, uint32_t& map) {
+    map = 0xFu;
+    return live_tile(p, I.kind, I.T, jj++, I.sink_end, I.win_lo, I.csr_beg);
+  }
+};
+template <bool kB64>
+__device__ __forceinline__ Walk<kB64> start_walk(const PatternDev& p, const Item& I, int H_kv) {
+  Walk<kB64> k;
   k.jj = 0;
-  k.w.a0 = k.w.e0 = k.w.a1 = k.w.e1 = 0;
-  if (bs64_kind(p, I.kind)) bs64_rows(p, H_kv, I.b, I.h, I.T, k.w);
+  if constexpr (kB64) {
+    k.w.a0 = k.w.e0 = k.w.a1 = k.w.e1 = 0;
+    if (bs64_kind(p, I.kind)) bs64_rows(p, H_kv, I.b, I.h, I.T, k.w);
+  }
   return k;
 }
 
@@ -323,6 +336,7 @@ __device__ __forceinline__ void store_p_row(uint32_t p_tile, int row, const uint
   }
 }
 
+template <bool kB64>
 __global__ void __launch_bounds__(kThreads, 1)
 hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o,
@@ -396,7 +410,7 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         // Ring order = MMA order: K0, then per tile jj: K(jj+1), V(jj).  The K walk runs
         // one tile ahead of the V walk.
-        Walk kw = start_walk(p, I, H_kv), vw = start_walk(p, I, H_kv);
+        Walk<kB64> kw = start_walk<kB64>(p, I, H_kv), vw = start_walk<kB64>(p, I, H_kv);
         uint32_t map;
         for (int jj = 0; jj < I.n && ok; ++jj) {
           if (jj == 0) ok = load_tile(&tm_k, I.h, max(0, kw.next(p, I, map)), I.b);
@@ -488,8 +502,8 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       const int i_out = I.t * BM + row;    // row of q and o in this call
       const int kind_el = I.kind == EA_STREAMING ? EA_STREAMING : EA_FULL;
       float m_ref = -INFINITY, l = 0.f;
-      const bool blk64 = p.block == 64 && (I.kind == EA_BLOCK_SPARSE || I.kind == EA_STREAMING_BLOCKS);
-      Walk walk = start_walk(p, I, H_kv);
+      const bool blk64 = kB64 && p.block == 64 && (I.kind == EA_BLOCK_SPARSE || I.kind == EA_STREAMING_BLOCKS);
+      Walk<kB64> walk = start_walk<kB64>(p, I, H_kv);
       for (int jj = 0; jj < I.n; ++jj) {
         uint32_t map;
         const int ct = walk.next(p, I, map);
@@ -515,7 +529,7 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         float f;
         if (ct < 0) {
           f = softmax_tile<1>(x, -1, 0, 0, p.scale_log2, m_ref, l, pk);
-        } else if (blk64) {   // 64x64 blocks: the key halves this warp's query half may read
+        } else if (kB64 && blk64) {   // 64x64 blocks: the key halves this warp's query half may read
           const int hb = (int)half_bits(p, I.kind, I.T, ct, row >> 6, map);
           if (hb == 3 && ct < I.T)
             f = softmax_tile<0>(x, 0, 0, 0, p.scale_log2, m_ref, l, pk);
@@ -646,7 +660,8 @@ ea_status launch_attn_tc(const void* q, const void* k, const void* v, void* o, c
     return EA_ERR_CUDA;
   const long long n_items = (long long)B * H_kv * pat.n_qt * n_pairs(H_q, H_kv);
   const int grid = (int)std::min<long long>(n_items, sm_count());
-  auto kern = hybrid_attn_tc_kernel;
+  // The block-64 instance carries the 64x64 block walk; block-128 patterns use the lean one.
+  auto kern = pat.block == 64 ? hybrid_attn_tc_kernel<true> : hybrid_attn_tc_kernel<false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) != cudaSuccess)
     return EA_ERR_CUDA;
   char* ws = static_cast<char*>(workspace);

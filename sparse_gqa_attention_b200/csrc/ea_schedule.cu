@@ -32,53 +32,62 @@ __device__ __forceinline__ void decode_item(int x, int np, int n_qt, int H_kv, i
   b = r / H_kv;
 }
 
-__device__ __forceinline__ int item_cost(const PatternDev& p, const int32_t* head_mode, int H_kv, int G,
-                                         int b, int h, int t, int pr, int n_bins) {
+// One thread per (b, h_kv, query tile of the call): the tile's live key tiles, and the
+// device checks of head_mode and of the tile's block-layout rows.
+__global__ void __launch_bounds__(256)
+tile_cost_kernel(const int32_t* __restrict__ head_mode, PatternDev p, int B, int H_kv, uint32_t* __restrict__ hdr,
+                 int* __restrict__ cost) {
+  const int x = blockIdx.x * blockDim.x + threadIdx.x;
+  if (x >= B * H_kv * p.n_qt) return;
+  const int tl = x % p.n_qt, bh = x / p.n_qt, h = bh % H_kv, b = bh / H_kv;
+  const int t = tl + p.q_tile0;   // global query tile
+  uint32_t bad = 0;
+  const int m = head_mode[b * H_kv + h];
+  if (m != 0 && m != 1) bad |= kStatusBadMode;
   const int kind = head_kind(p, head_mode, H_kv, b, h);
-  const int n = n_live_tiles(p, kind, H_kv, b, h, t);
+  if (kind == EA_BLOCK_SPARSE) {   // the tile's CSR rows (1 at block 128, 2 at 64)
+    const int per = kTile / p.block;
+    for (int u = 0; u < per; ++u) {
+      const int qb = t * per + u;
+      if (qb >= p.n_qb) break;
+      const long long r = ((long long)b * H_kv + h) * p.n_qb + qb;
+      const long long a0 = p.row_ptr[r], a1 = p.row_ptr[r + 1];
+      if (a0 < 0 || a1 < a0 || a1 > p.nnz || a1 == a0) {
+        bad |= kStatusBadLayout;
+      } else {
+        int prev = -1;
+        for (long long e = a0; e < a1; ++e) {
+          const int c = p.cols[e];
+          if (c <= prev || c > qb) bad |= kStatusBadLayout;
+          prev = c;
+        }
+        if (prev != qb) bad |= kStatusBadLayout;
+      }
+    }
+  }
+  cost[x] = n_live_tiles(p, kind, H_kv, b, h, t);
+  if (bad) atomicOr(hdr + kWsStatus / 4, bad);
+}
+
+__device__ __forceinline__ int item_cost(const int* cost, int n_qt, int H_kv, int G, int b, int h, int tl, int pr,
+                                         int n_bins) {
   const int heads = min(2, G - 2 * pr);
-  return min(n * heads, n_bins - 1);
+  return min(cost[(b * H_kv + h) * n_qt + tl] * heads, n_bins - 1);
 }
 
 __global__ void __launch_bounds__(kSchedThreads)
-schedule_kernel(const int32_t* __restrict__ head_mode, PatternDev p, int H_kv, int G, int np, int n_items,
-                int n_bins, uint32_t* __restrict__ hdr, int4* __restrict__ items) {
+schedule_kernel(const int* __restrict__ cost, PatternDev p, int H_kv, int G, int np, int n_items, int n_bins,
+                uint32_t* __restrict__ hdr, int4* __restrict__ items) {
   __shared__ int bins[kMaxBins];
   __shared__ int part[kSchedThreads];
   const int tid = threadIdx.x;
   for (int i = tid; i < n_bins; i += kSchedThreads) bins[i] = 0;
   __syncthreads();
-  uint32_t bad = 0;
   for (int x = tid; x < n_items; x += kSchedThreads) {
     int b, h, tl, pr;
     decode_item(x, np, p.n_qt, H_kv, b, h, tl, pr);
-    const int t = tl + p.q_tile0;   // global query tile
-    const int m = head_mode[b * H_kv + h];
-    if (m != 0 && m != 1) bad |= kStatusBadMode;
-    const int kind = head_kind(p, head_mode, H_kv, b, h);
-    if (kind == EA_BLOCK_SPARSE && pr == 0) {   // the tile's CSR rows (1 at block 128, 2 at 64)
-      const int per = kTile / p.block;
-      for (int u = 0; u < per; ++u) {
-        const int qb = t * per + u;
-        if (qb >= p.n_qb) break;
-        const long long r = ((long long)b * H_kv + h) * p.n_qb + qb;
-        const long long a0 = p.row_ptr[r], a1 = p.row_ptr[r + 1];
-        if (a0 < 0 || a1 < a0 || a1 > p.nnz || a1 == a0) {
-          bad |= kStatusBadLayout;
-        } else {
-          int prev = -1;
-          for (long long e = a0; e < a1; ++e) {
-            const int c = p.cols[e];
-            if (c <= prev || c > qb) bad |= kStatusBadLayout;
-            prev = c;
-          }
-          if (prev != qb) bad |= kStatusBadLayout;
-        }
-      }
-    }
-    atomicAdd(&bins[item_cost(p, head_mode, H_kv, G, b, h, t, pr, n_bins)], 1);
+    atomicAdd(&bins[item_cost(cost, p.n_qt, H_kv, G, b, h, tl, pr, n_bins)], 1);
   }
-  if (bad) atomicOr(hdr + kWsStatus / 4, bad);
   // (items store the local query tile; the attention kernels add q_tile0)
   __syncthreads();
   // Exclusive scan of the bins in descending cost order: bins[c] <- items costing more than c.
@@ -105,7 +114,7 @@ schedule_kernel(const int32_t* __restrict__ head_mode, PatternDev p, int H_kv, i
   for (int x = tid; x < n_items; x += kSchedThreads) {
     int b, h, tl, pr;
     decode_item(x, np, p.n_qt, H_kv, b, h, tl, pr);
-    const int pos = atomicAdd(&bins[item_cost(p, head_mode, H_kv, G, b, h, tl + p.q_tile0, pr, n_bins)], 1);
+    const int pos = atomicAdd(&bins[item_cost(cost, p.n_qt, H_kv, G, b, h, tl, pr, n_bins)], 1);
     items[pos] = make_int4(b, h, tl, pr);
   }
   if (tid == 0) hdr[kWsNItems / 4] = (uint32_t)n_items;
@@ -162,9 +171,14 @@ int n_pairs(int H_q, int H_kv) { return (H_q / H_kv + 1) / 2; }
 
 static size_t items_offset(int B) { return kWsHeader + ((size_t)B * 4 + 255) / 256 * 256; }
 
-size_t attn_workspace_bytes(int B, int S, int H_q, int H_kv) {
+// Workspace: header | per-sample sparse-head counts | int4 work items | int32 tile costs.
+static size_t costs_offset(int B, int S, int H_q, int H_kv) {
   const size_t n_items = (size_t)B * H_kv * cdiv(S, kTile) * n_pairs(H_q, H_kv);
   return items_offset(B) + n_items * sizeof(int4);
+}
+
+size_t attn_workspace_bytes(int B, int S, int H_q, int H_kv) {
+  return costs_offset(B, S, H_q, H_kv) + ((size_t)B * H_kv * cdiv(S, kTile) * 4 + 255) / 256 * 256;
 }
 
 ea_status launch_schedule(const int32_t* head_mode, const PatternDev& pat, int B, int S, int H_q, int H_kv,
@@ -174,7 +188,11 @@ ea_status launch_schedule(const int32_t* head_mode, const PatternDev& pat, int B
   if (n_items > (1LL << 30)) return EA_ERR_UNSUPPORTED;
   const int n_bins = min(kMaxBins, 2 * (pat.n_qt + pat.q_tile0) + 1);
   char* ws = static_cast<char*>(workspace);
-  schedule_kernel<<<1, kSchedThreads, 0, st>>>(head_mode, pat, H_kv, G, np, (int)n_items, n_bins,
+  int* cost = reinterpret_cast<int*>(ws + costs_offset(B, S, H_q, H_kv));
+  const int n_bt = B * H_kv * pat.n_qt;
+  tile_cost_kernel<<<cdiv(n_bt, 256), 256, 0, st>>>(head_mode, pat, B, H_kv, reinterpret_cast<uint32_t*>(ws), cost);
+  if (cudaGetLastError() != cudaSuccess) return EA_ERR_CUDA;
+  schedule_kernel<<<1, kSchedThreads, 0, st>>>(cost, pat, H_kv, G, np, (int)n_items, n_bins,
                                                reinterpret_cast<uint32_t*>(ws),
                                                reinterpret_cast<int4*>(ws + items_offset(B)));
   return cudaGetLastError() == cudaSuccess ? EA_OK : EA_ERR_CUDA;

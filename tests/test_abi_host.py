@@ -30,10 +30,11 @@ def test_status_strings(lib):
 
 
 def test_workspace_sizes(lib):
-    # 2 pairs x 8 KV heads x 256 query tiles of 16-byte items, after a 256 + 256 byte header.
-    assert abi.ea_attn_workspace_size(1, 32768, 32, 8) == 512 + 8 * 256 * 2 * 16
+    # 2 pairs x 8 KV heads x 256 query tiles of 16-byte items, after a 256 + 256 byte header,
+    # then one int32 live-tile count per (KV head, query tile).
+    assert abi.ea_attn_workspace_size(1, 32768, 32, 8) == 512 + 8 * 256 * 2 * 16 + 8 * 256 * 4
     assert abi.ea_attn_workspace_size(1, 100, 7, 2) == 0          # H_q not a multiple of H_kv
-    assert abi.ea_attn_workspace_size(1, 65536, 28, 4) == 512 + 4 * 512 * 4 * 16
+    assert abi.ea_attn_workspace_size(1, 65536, 28, 4) == 512 + 4 * 512 * 4 * 16 + 4 * 512 * 4
     n = abi.ea_router_workspace_size(1, 32768, 4096, 8, 128, 100)
     assert n > 4096 * 4 and n % 256 == 0
 
