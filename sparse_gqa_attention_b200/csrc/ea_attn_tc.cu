@@ -122,6 +122,7 @@ __device__ __forceinline__ int item_index(int it, int cta, int ncta) {
   return it * ncta + ((it & 1) ? (ncta - 1 - cta) : cta);
 }
 
+template <bool kB64>
 __device__ __forceinline__ Item load_item(const int4* items, int idx, const PatternDev& p,
                                           const int32_t* head_mode, int H_kv, int G) {
   const int4 w = items[idx];
@@ -135,7 +136,7 @@ __device__ __forceinline__ Item load_item(const int4* items, int idx, const Patt
   if (is_streaming(I.kind)) {
     stream_ranges(p, I.kind, I.T, I.sink_end, I.win_lo);
     I.n = I.sink_end + max(0, I.T - I.win_lo + 1);
-  } else if (bs64_kind(p, I.kind)) {
+  } else if (kB64 && bs64_kind(p, I.kind)) {
     I.n = n_live_tiles(p, I.kind, H_kv, I.b, I.h, I.T);
   } else if (I.kind == EA_BLOCK_SPARSE) {
     long long a, e;
@@ -394,7 +395,7 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       for (int it = 0; ok; ++it) {
         const int idx = item_index(it, blockIdx.x, gridDim.x);
         if (idx >= n_items) break;
-        const Item I = load_item(items, idx, p, head_mode, H_kv, G);
+        const Item I = load_item<kB64>(items, idx, p, head_mode, H_kv, G);
         if (I.n == 0) continue;
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
@@ -437,7 +438,7 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       for (int it = 0; ok; ++it) {
         const int idx = item_index(it, blockIdx.x, gridDim.x);
         if (idx >= n_items) break;
-        const Item I = load_item(items, idx, p, head_mode, H_kv, G);
+        const Item I = load_item<kB64>(items, idx, p, head_mode, H_kv, G);
         if (I.n == 0) continue;
         ok = wait(c, c.bar(B_QFULL + 0), q_use[0] & 1);
         ++q_use[0];
@@ -496,7 +497,7 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     for (int it = 0; ok; ++it) {
       const int idx = item_index(it, blockIdx.x, gridDim.x);
       if (idx >= n_items) break;
-      const Item I = load_item(items, idx, p, head_mode, H_kv, G);
+      const Item I = load_item<kB64>(items, idx, p, head_mode, H_kv, G);
       if (I.n == 0 || (s == 1 && !I.two)) continue;
       const int i = I.T * BM + row;        // query position in the sequence
       const int i_out = I.t * BM + row;    // row of q and o in this call

@@ -14,7 +14,8 @@
 //
 // Kernels, in stream order:
 //   xattn_plan_kernel    the (b, h_q) whose KV head is BLOCK_SPARSE under head_mode;
-//   xattn_score_kernel   R tile by tile on the tensor cores (tcgen05, TMEM accumulators,
+//   xattn_score_kernel   R on the tensor cores, 128 reduced rows x 256 reduced columns per
+//                        MMA (one q chunk feeds two key tiles; tcgen05, TMEM accumulators,
 //                        TMA 5-D maps that split the sequence into (reduced row, m)), and
 //                        per reduced row and 128-key block the partial softmax sums
 //                        relative to the tile's row maximum;
@@ -38,11 +39,13 @@ namespace {
 using namespace sm100;
 
 constexpr int XT = 128;                       // reduced rows (and columns) per tile
-constexpr int XNS = 6;                        // K-chunk stages
-constexpr uint32_t kChunkBytes = 16384;       // 128 rows x 64 bf16
+constexpr int XN = 256;                       // reduced key columns per MMA: a pair of tiles
+constexpr int XNS = 4;                        // K-chunk stages
+constexpr uint32_t kChunkBytes = 16384;       // 128 rows x 64 bf16 (q chunk)
+constexpr uint32_t kBChunkBytes = 32768;      // 256 rows x 64 bf16 (k chunk)
 constexpr uint32_t X_OFF_A = 0;
 constexpr uint32_t X_OFF_B = XNS * kChunkBytes;
-constexpr uint32_t X_OFF_BAR = 2 * XNS * kChunkBytes;
+constexpr uint32_t X_OFF_BAR = XNS * (kChunkBytes + kBChunkBytes);
 enum : int { X_FULL = 0, X_EMPTY = XNS, X_AFULL = 2 * XNS, X_AEMPTY = X_AFULL + 2, X_FIN = X_AEMPTY + 2,
              X_NBAR = X_FIN + 1 };
 constexpr uint32_t X_OFF_TMEM = X_OFF_BAR + X_NBAR * 8;
@@ -50,8 +53,8 @@ constexpr uint32_t X_OFF_ABORT = X_OFF_TMEM + 4;
 constexpr uint32_t kXSmemBytes = X_OFF_ABORT + 4 + 1024;   // + slack to align the base to 1024
 static_assert(kXSmemBytes <= 232448, "shared memory beyond the 227 KB a CTA may use");
 constexpr int kXThreads = 192;                // warp 0 TMA, warp 1 TMEM + MMA, warps 2-5 epilogue
-constexpr uint32_t kXTmemCols = 256;          // two 128-column accumulators
-constexpr uint32_t IDESC_X = idesc_bf16(128, 128, false);
+constexpr uint32_t kXTmemCols = 512;          // two 256-column accumulators
+constexpr uint32_t IDESC_X = idesc_bf16(128, XN, false);
 constexpr unsigned long long kXWaitLimitNs = 2000000000ull;
 
 constexpr int kSelThreads = 256;
@@ -235,15 +238,15 @@ xattn_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const int idx = x_item_index(it, blockIdx.x, gridDim.x);
         if (idx >= n_work) break;
         const XItem I = x_item(plan, idx, n_live, n_rt, H_q, G);
-        for (int ct = 0; ct <= I.r && ok; ++ct) {
+        for (int pp = 0; pp <= I.r / 2 && ok; ++pp) {   // key tiles 2pp, 2pp+1
           for (int q = 0; q < NCH; ++q) {
             const int s = ch % XNS, m = q >> 1, half = q & 1;
             ok = xwait(c, c.bar(X_EMPTY + s), ((ch / XNS) & 1) ^ 1);
             if (!ok) break;
-            mbar_expect_tx(c.bar(X_FULL + s), 2 * kChunkBytes);
+            mbar_expect_tx(c.bar(X_FULL + s), kChunkBytes + kBChunkBytes);
             tma_load_5d(base + X_OFF_A + s * kChunkBytes, &tm_q, c.bar(X_FULL + s), 64 * half, I.h, m, XT * I.r, I.b);
-            tma_load_5d(base + X_OFF_B + s * kChunkBytes, &tm_k, c.bar(X_FULL + s), 64 * half, I.hk, ST - 1 - m,
-                        XT * ct, I.b);
+            tma_load_5d(base + X_OFF_B + s * kBChunkBytes, &tm_k, c.bar(X_FULL + s), 64 * half, I.hk, ST - 1 - m,
+                        XN * pp, I.b);
             ++ch;
           }
         }
@@ -262,7 +265,7 @@ xattn_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const int idx = x_item_index(it, blockIdx.x, gridDim.x);
         if (idx >= n_work) break;
         const XItem I = x_item(plan, idx, n_live, n_rt, H_q, G);
-        for (int ct = 0; ct <= I.r && ok; ++ct) {
+        for (int pp = 0; pp <= I.r / 2 && ok; ++pp) {
           const int a = tile & 1;
           ok = xwait(c, c.bar(X_AEMPTY + a), ((tile >> 1) & 1) ^ 1);
           if (!ok) break;
@@ -272,10 +275,10 @@ xattn_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             ok = xwait(c, c.bar(X_FULL + s), (ch / XNS) & 1);
             if (!ok) break;
             fence_after_sync();
-            const uint32_t at = base + X_OFF_A + s * kChunkBytes, bt = base + X_OFF_B + s * kChunkBytes;
+            const uint32_t at = base + X_OFF_A + s * kChunkBytes, bt = base + X_OFF_B + s * kBChunkBytes;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_ss(tmem + 128u * a, x_desc(at, kk), x_desc(bt, kk), IDESC_X, (q > 0 || kk > 0) ? 1u : 0u);
+              mma_ss(tmem + (uint32_t)XN * a, x_desc(at, kk), x_desc(bt, kk), IDESC_X, (q > 0 || kk > 0) ? 1u : 0u);
             commit(c.bar(X_EMPTY + s));
             ++ch;
           }
@@ -301,32 +304,39 @@ xattn_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const XItem I = x_item(plan, idx, n_live, n_rt, H_q, G);
       const int i = XT * I.r + row;
       const size_t rrow = (size_t)I.bh * n_red + i;
-      for (int ct = 0; ct <= I.r; ++ct) {
+      for (int pp = 0; pp <= I.r / 2; ++pp) {
         const int a = tile & 1;
         ok = xwait(c, c.bar(X_AFULL + a), (tile >> 1) & 1);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         ++tile;
         fence_after_sync();
-        float x[XT];
-        {
-          uint32_t rr[XT];
+        for (int hf = 0; hf < 2; ++hf) {   // key tiles 2pp and 2pp+1 (the second may lie past the diagonal)
+          const int ct = 2 * pp + hf;
+          float x[XT];
+          {
+            uint32_t rr[XT];
 #pragma unroll
-          for (int q4 = 0; q4 < XT / 32; ++q4) tmem_ld32(lane_addr + 128u * a + 32 * q4, rr + 32 * q4);
-          tmem_ld_wait();
+            for (int q4 = 0; q4 < XT / 32; ++q4)
+              tmem_ld32(lane_addr + (uint32_t)XN * a + 128u * hf + 32 * q4, rr + 32 * q4);
+            tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < XT; ++e) x[e] = __uint_as_float(rr[e]);
-        }
-        fence_before_sync();
-        mbar_arrive(c.bar(X_AEMPTY + a));
-        if (i < n_red) {
-          float sg[ST];
-          const float ms = ct < I.r ? x_row_tile<ST, false>(x, XT - 1, sl2, sg) : x_row_tile<ST, true>(x, row, sl2, sg);
-          float* sp = s_part + rrow * pitch + ct * ST;
+            for (int e = 0; e < XT; ++e) x[e] = __uint_as_float(rr[e]);
+          }
+          if (hf == 1) {   // the accumulator is free once both halves are in registers
+            fence_before_sync();
+            mbar_arrive(c.bar(X_AEMPTY + a));
+          }
+          if (i < n_red && ct <= I.r) {
+            float sg[ST];
+            const float ms =
+                ct < I.r ? x_row_tile<ST, false>(x, XT - 1, sl2, sg) : x_row_tile<ST, true>(x, row, sl2, sg);
+            float* sp = s_part + rrow * pitch + ct * ST;
 #pragma unroll
-          for (int g = 0; g < ST; g += 4)
-            *reinterpret_cast<float4*>(sp + g) = make_float4(sg[g], sg[g + 1], sg[g + 2], sg[g + 3]);
-          m_part[rrow * n_rt + ct] = ms;
+            for (int g = 0; g < ST; g += 4)
+              *reinterpret_cast<float4*>(sp + g) = make_float4(sg[g], sg[g + 1], sg[g + 2], sg[g + 3]);
+            m_part[rrow * n_rt + ct] = ms;
+          }
         }
       }
     }
@@ -577,14 +587,15 @@ XEncodeFn x_encode_fn() {
 }
 
 // [B, S, H, 128] bf16 viewed as 5-D (d, H, st, S/st, B): coordinate (x, h, m, i, b) is
-// element x of head h at sequence row i*st + m.  Box: 64 columns x 1 x 1 x 128 reduced rows.
-bool make_map5(CUtensorMap* m, const void* ptr, int B, int S, int H, int st) {
+// element x of head h at sequence row i*st + m.  Box: 64 columns x 1 x 1 x box_rows reduced rows
+// (128 for q, 256 for k).
+bool make_map5(CUtensorMap* m, const void* ptr, int B, int S, int H, int st, int box_rows) {
   XEncodeFn fn = x_encode_fn();
   if (!fn) return false;
   const cuuint64_t row = (cuuint64_t)H * 128 * 2;
   const cuuint64_t dims[5] = {128, (cuuint64_t)H, (cuuint64_t)st, (cuuint64_t)(S / st), (cuuint64_t)B};
   const cuuint64_t strides[4] = {256, row, row * st, row * S};
-  const cuuint32_t box[5] = {64, 1, 1, (cuuint32_t)XT, 1};
+  const cuuint32_t box[5] = {64, 1, 1, (cuuint32_t)box_rows, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -604,7 +615,7 @@ ea_status launch_st(const void* q, const void* k, const int32_t* head_mode, cons
                     cudaStream_t st) {
   const XLayout L = x_layout(B, S, H_q, H_kv, ST);
   CUtensorMap mq, mk;
-  if (!make_map5(&mq, q, B, S, H_q, ST) || !make_map5(&mk, k, B, S, H_kv, ST)) return EA_ERR_CUDA;
+  if (!make_map5(&mq, q, B, S, H_q, ST, XT) || !make_map5(&mk, k, B, S, H_kv, ST, XN)) return EA_ERR_CUDA;
   char* ws = static_cast<char*>(workspace);
   uint32_t* hdr = reinterpret_cast<uint32_t*>(ws);
   int* plan = reinterpret_cast<int*>(ws + L.plan);
