@@ -122,7 +122,6 @@ __device__ __forceinline__ int item_index(int it, int cta, int ncta) {
   return it * ncta + ((it & 1) ? (ncta - 1 - cta) : cta);
 }
 
-template <bool kB64>
 __device__ __forceinline__ Item load_item(const int4* items, int idx, const PatternDev& p,
                                           const int32_t* head_mode, int H_kv, int G) {
   const int4 w = items[idx];
@@ -136,8 +135,6 @@ __device__ __forceinline__ Item load_item(const int4* items, int idx, const Patt
   if (is_streaming(I.kind)) {
     stream_ranges(p, I.kind, I.T, I.sink_end, I.win_lo);
     I.n = I.sink_end + max(0, I.T - I.win_lo + 1);
-  } else if (kB64 && bs64_kind(p, I.kind)) {
-    I.n = n_live_tiles(p, I.kind, H_kv, I.b, I.h, I.T);
   } else if (I.kind == EA_BLOCK_SPARSE) {
     long long a, e;
     csr_row(p, H_kv, I.b, I.h, I.T, a, e);
@@ -147,45 +144,6 @@ __device__ __forceinline__ Item load_item(const int4* items, int idx, const Patt
     I.n = I.T + 1;
   }
   return I;
-}
-
-// Sequential walk over an item's live key tiles: the tile index (-1: nothing live) and,
-// for block-64 block-sparse heads, the 2x2 map of its live blocks (0xF otherwise).  The
-// block-64 state exists only in the kernel instance launched for block-64 patterns.
-template <bool kB64>
-struct Walk {
-  Bs64 w;
-  int jj;
-  __device__ __forceinline__ int next(const PatternDev& p, const Item& I, uint32_t& map) {
-    map = 0xFu;
-    int c;
-    if (bs64_kind(p, I.kind)) {
-      c = bs64_next(p, w, map);
-      if (c > I.T) c = -1;   // a block above the diagonal (malformed layout): skipped
-    } else {
-      c = live_tile(p, I.kind, I.T, jj, I.sink_end, I.win_lo, I.csr_beg);
-    }
-    ++jj;
-    return c;
-  }
-};
-template <>
-struct Walk<false> {
-  int jj;
-  __device__ __forceinline__ int next(const PatternDev& p, const Item& I, uint32_t& map) {
-    map = 0xFu;
-    return live_tile(p, I.kind, I.T, jj++, I.sink_end, I.win_lo, I.csr_beg);
-  }
-};
-template <bool kB64>
-__device__ __forceinline__ Walk<kB64> start_walk(const PatternDev& p, const Item& I, int H_kv) {
-  Walk<kB64> k;
-  k.jj = 0;
-  if constexpr (kB64) {
-    k.w.a0 = k.w.e0 = k.w.a1 = k.w.e1 = 0;
-    if (bs64_kind(p, I.kind)) bs64_rows(p, H_kv, I.b, I.h, I.T, k.w);
-  }
-  return k;
 }
 
 __device__ __forceinline__ uint64_t qk_desc(uint32_t tile, int kk) {
@@ -265,8 +223,7 @@ __device__ __forceinline__ void ex2_pair_fma(uint64_t t2, float& r0, float& r1) 
 
 // One 128-key tile of one query row: running max (raised only past kRescaleLog2),
 // row sum, and P = exp2(scale*log2e*s - max) as bf16 pairs in pk (pk[j] holds keys
-// 2j, 2j+1).  kMode 0: every key live; 1: causal rule; 2: streaming rule; 3: causal
-// rule within the enabled 64-key halves (block-64 kinds; sink_lim holds the bits).  Returns
+// 2j, 2j+1).  kMode 0: every key live; 1: causal rule; 2: streaming rule.  Returns
 // the factor O must be multiplied by (1 when the max was not raised).
 template <int kMode>
 __device__ __forceinline__ float softmax_tile(const float (&x)[BN], int lim, int sink_lim, int win_lim,
@@ -274,7 +231,6 @@ __device__ __forceinline__ float softmax_tile(const float (&x)[BN], int lim, int
   auto live = [&](int e) {
     if (kMode == 0) return true;
     if (kMode == 1) return e <= lim;
-    if (kMode == 3) return e <= lim && ((sink_lim >> (e >> 6)) & 1) != 0;   // sink_lim: key-half bits
     return e <= lim && (e < sink_lim || e > win_lim);
   };
   auto xm = [&](int e) { return live(e) ? x[e] : -INFINITY; };
@@ -337,7 +293,6 @@ __device__ __forceinline__ void store_p_row(uint32_t p_tile, int row, const uint
   }
 }
 
-template <bool kB64>
 __global__ void __launch_bounds__(kThreads, 1)
 hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o,
@@ -395,7 +350,7 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       for (int it = 0; ok; ++it) {
         const int idx = item_index(it, blockIdx.x, gridDim.x);
         if (idx >= n_items) break;
-        const Item I = load_item<kB64>(items, idx, p, head_mode, H_kv, G);
+        const Item I = load_item(items, idx, p, head_mode, H_kv, G);
         if (I.n == 0) continue;
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
@@ -409,14 +364,12 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           tma_load_4d(dst + kBoxBytes, &tm_q, c.bar(B_QFULL + s), 64, h_q, I.t * BM, I.b);
           ++q_use[s];
         }
-        // Ring order = MMA order: K0, then per tile jj: K(jj+1), V(jj).  The K walk runs
-        // one tile ahead of the V walk.
-        Walk<kB64> kw = start_walk<kB64>(p, I, H_kv), vw = start_walk<kB64>(p, I, H_kv);
-        uint32_t map;
+        // Ring order = MMA order: K0, then per tile jj: K(jj+1), V(jj).
+        auto tile = [&](int jj) { return max(0, live_tile(p, I.kind, I.T, jj, I.sink_end, I.win_lo, I.csr_beg)); };
         for (int jj = 0; jj < I.n && ok; ++jj) {
-          if (jj == 0) ok = load_tile(&tm_k, I.h, max(0, kw.next(p, I, map)), I.b);
-          if (ok && jj + 1 < I.n) ok = load_tile(&tm_k, I.h, max(0, kw.next(p, I, map)), I.b);
-          if (ok) ok = load_tile(&tm_v, I.h, max(0, vw.next(p, I, map)), I.b);
+          if (jj == 0) ok = load_tile(&tm_k, I.h, tile(0), I.b);
+          if (ok && jj + 1 < I.n) ok = load_tile(&tm_k, I.h, tile(jj + 1), I.b);
+          if (ok) ok = load_tile(&tm_v, I.h, tile(jj), I.b);
         }
       }
       // Drain: the last copy armed on every barrier has landed before the CTA exits.
@@ -438,7 +391,7 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       for (int it = 0; ok; ++it) {
         const int idx = item_index(it, blockIdx.x, gridDim.x);
         if (idx >= n_items) break;
-        const Item I = load_item<kB64>(items, idx, p, head_mode, H_kv, G);
+        const Item I = load_item(items, idx, p, head_mode, H_kv, G);
         if (I.n == 0) continue;
         ok = wait(c, c.bar(B_QFULL + 0), q_use[0] & 1);
         ++q_use[0];
@@ -497,17 +450,14 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     for (int it = 0; ok; ++it) {
       const int idx = item_index(it, blockIdx.x, gridDim.x);
       if (idx >= n_items) break;
-      const Item I = load_item<kB64>(items, idx, p, head_mode, H_kv, G);
+      const Item I = load_item(items, idx, p, head_mode, H_kv, G);
       if (I.n == 0 || (s == 1 && !I.two)) continue;
       const int i = I.T * BM + row;        // query position in the sequence
       const int i_out = I.t * BM + row;    // row of q and o in this call
       const int kind_el = I.kind == EA_STREAMING ? EA_STREAMING : EA_FULL;
       float m_ref = -INFINITY, l = 0.f;
-      const bool blk64 = kB64 && p.block == 64 && (I.kind == EA_BLOCK_SPARSE || I.kind == EA_STREAMING_BLOCKS);
-      Walk<kB64> walk = start_walk<kB64>(p, I, H_kv);
       for (int jj = 0; jj < I.n; ++jj) {
-        uint32_t map;
-        const int ct = walk.next(p, I, map);
+        const int ct = live_tile(p, I.kind, I.T, jj, I.sink_end, I.win_lo, I.csr_beg);
         ok = wait(c, c.bar(B_SFULL + s), s_cnt & 1);
         ok = __all_sync(0xffffffffu, ok);
         ++s_cnt;
@@ -530,12 +480,6 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         float f;
         if (ct < 0) {
           f = softmax_tile<1>(x, -1, 0, 0, p.scale_log2, m_ref, l, pk);
-        } else if (kB64 && blk64) {   // 64x64 blocks: the key halves this warp's query half may read
-          const int hb = (int)half_bits(p, I.kind, I.T, ct, row >> 6, map);
-          if (hb == 3 && ct < I.T)
-            f = softmax_tile<0>(x, 0, 0, 0, p.scale_log2, m_ref, l, pk);
-          else
-            f = softmax_tile<3>(x, i - ct * BN, hb, 0, p.scale_log2, m_ref, l, pk);
         } else if (tile_needs_mask(p, I.kind, I.T, ct)) {
           const int lim = i - ct * BN;
           if (kind_el == EA_STREAMING)
@@ -656,13 +600,13 @@ int sm_count() {
 ea_status launch_attn_tc(const void* q, const void* k, const void* v, void* o, const int32_t* head_mode,
                          const PatternDev& pat, int B, int S, int S_k, int H_q, int H_kv, void* workspace,
                          cudaStream_t st) {
+  if (pat.block == 64) return launch_attn_tc64(q, k, v, o, head_mode, pat, B, S, S_k, H_q, H_kv, workspace, st);
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, B, S, H_q) || !make_map(&mk, k, B, S_k, H_kv) || !make_map(&mv, v, B, S_k, H_kv))
     return EA_ERR_CUDA;
   const long long n_items = (long long)B * H_kv * pat.n_qt * n_pairs(H_q, H_kv);
   const int grid = (int)std::min<long long>(n_items, sm_count());
-  // The block-64 instance carries the 64x64 block walk; block-128 patterns use the lean one.
-  auto kern = pat.block == 64 ? hybrid_attn_tc_kernel<true> : hybrid_attn_tc_kernel<false>;
+  auto kern = hybrid_attn_tc_kernel;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) != cudaSuccess)
     return EA_ERR_CUDA;
   char* ws = static_cast<char*>(workspace);

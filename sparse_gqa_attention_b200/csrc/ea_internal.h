@@ -27,6 +27,10 @@ ea_status launch_attn_simt(const float* q, const float* k, const float* v, float
 ea_status launch_attn_tc(const void* q, const void* k, const void* v, void* o, const int32_t* head_mode,
                          const PatternDev& pat, int B, int S, int S_k, int H_q, int H_kv, void* workspace,
                          cudaStream_t st);
+// Block-64 layouts (ea_attn_tc64.cu); launch_attn_tc forwards to it.
+ea_status launch_attn_tc64(const void* q, const void* k, const void* v, void* o, const int32_t* head_mode,
+                           const PatternDev& pat, int B, int S, int S_k, int H_q, int H_kv, void* workspace,
+                           cudaStream_t st);
 
 // XAttention block selection (ea_xattn.cu).
 bool xattn_shape_ok(int S, int H_q, int H_kv, int stride);
