@@ -257,17 +257,18 @@ __device__ __forceinline__ float softmax_tile(const float (&x)[BN], int lim, int
 #pragma unroll
   for (int e = 0; e < BN; e += 2) {
     const uint64_t t2 = f2_fma(f2_pack(x[e], x[e + 1]), scale2, nsub2);
-    float e0, e1;
+    float p0, p1;
     if (kPolyEvery > 0 && (e / 2) % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
+      float e0, e1;
       ex2_pair_fma(t2, e0, e1);
-    } else {
+      p0 = live(e) ? e0 : 0.f;
+      p1 = live(e + 1) ? e1 : 0.f;
+    } else {   // dead keys skip the MUFU (a whole warp past the diagonal skips it)
       float t0, t1;
       f2_unpack(t2, t0, t1);
-      e0 = ex2(t0);
-      e1 = ex2(t1);
+      p0 = live(e) ? ex2(t0) : 0.f;
+      p1 = live(e + 1) ? ex2(t1) : 0.f;
     }
-    const float p0 = live(e) ? e0 : 0.f;
-    const float p1 = live(e + 1) ? e1 : 0.f;
     l2 = f2_add(l2, f2_pack(p0, p1));
     pk[e / 2] = pack_bf16x2(p0, p1);
   }
