@@ -41,6 +41,7 @@ ATTN_TRAFFIC = {  # source hash -> {workload: bytes per launch}
     "0296169ffe64f919": {"llama3-8b-s32k-streaming": 588227584 + 242138624},
     "7f7dafa317af8ef7": {"llama3-8b-s32k-streaming": 592338944 + 243713536},
     "c9ec1a166bddf719": {"llama3-8b-s32k-streaming": 572987648 + 234234880},
+    "d295b6f17472de2e": {"llama3-8b-s32k-streaming": 581203968 + 235314688},
 }
 
 def attn_source_hash():
