@@ -329,8 +329,8 @@ def run_cuda(args):
             "router_roofline": router_full,
             **({"xattn_roofline": xattn_line} if xattn_line else {}),
             "e2e": e2e,
-            # router 3 + (XAttention 5) + schedule 2 + attention 1 + sparsity 1 per step
-            "gpu_launches": (12 if xattn else 7) * args.steps,
+            # router 7 + (XAttention 5) + schedule 2 + attention 1 + sparsity 1 per step
+            "gpu_launches": (16 if xattn else 11) * args.steps,
             "clocks": clk.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -8,10 +8,14 @@
 // Kernels (all fp32 arithmetic, fixed summation orders, so results are reproducible):
 //   pool_partial   HBM-bound streaming reduction of the pooled hidden rows: 16-byte
 //                  loads, 8 in flight per thread, one partial sum per (split, b, column).
-//   project        one CTA per 64 rows of W_k: finishes the pooled mean of its rows,
+//   project        one CTA per 32 rows of W_k: finishes the pooled mean of its rows,
 //                  then the partial key projections of those rows for every column.
-//   router_mlp     one CTA per (KV head, sample): sums the projection partials of its
-//                  head, task MLP, router MLP on [p; tau], output row, threshold.
+//   proj_reduce    p[b][h*d + c] = sum over the row chunks of the partial projections.
+//   mlp_layer x3   the task MLP's two layers and the router MLP, each a batched GEMV over
+//                  all (sample, KV head) vectors (the MLP weights are shared by the heads):
+//                  one warp per output row, the row held in registers, every vector of
+//                  the batch streamed past it.
+//   router_out     the head's output row, bias and threshold (one warp per (b, h)).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
@@ -86,7 +90,7 @@ pool_partial_kernel(const T* __restrict__ hidden, int S, int D, int n_rows, int 
   }
 }
 
-constexpr int kProjRows = 64;      // rows of W_k per projection CTA
+constexpr int kProjRows = 32;      // rows of W_k per projection CTA
 constexpr int kProjThreads = 256;
 constexpr int kProjB = 4;          // samples per pass over a W_k chunk
 
@@ -105,7 +109,7 @@ __device__ __forceinline__ void fma_vec(float* acc, uint4 raw, float x) {
   }
 }
 
-// grid (ceil(D / kProjRows)).  For rows [r0, r0 + 64) of W_k:
+// grid (ceil(D / kProjRows)).  For rows [r0, r0 + kProjRows) of W_k:
 //   hbar[b][r] = (sum over splits of the pooling partial sums) / n_rows      (fixed order)
 //   pp[chunk][b][n] = sum_{r in chunk} W_k[r, n] * hbar[b][r]   for every column n < N = H_kv*d
 template <typename T>
@@ -200,9 +204,8 @@ project_kernel(const float* __restrict__ partial, int n_splits, int B, int D, fl
   }
 }
 
-constexpr int kMlpThreads = 512;
+constexpr int kMlpThreads = 256;   // 8 warps, one output row each
 constexpr int kMlpWarps = kMlpThreads / 32;
-constexpr int kGemvRows = 8;       // rows per warp per pass: their loads are issued together
 
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
@@ -210,85 +213,73 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-// y[r] = act(W[r, :] . x + bias[r]) for r < rows (W row-major fp32, cols % 4 == 0, x in shared
-// memory).  Each warp takes kGemvRows rows per pass; a lane reads float4s at columns
-// 4*lane + 128*k, so all loads of a pass are in flight together.
+// p[i] = sum over the row chunks of pp[chunk][i] (fixed order), i < B * H_kv * d.
+__global__ void __launch_bounds__(256)
+proj_reduce_kernel(const float* __restrict__ pp, int n_chunks, int total, float* __restrict__ p) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= total) return;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  int ch = 0;
+  for (; ch + 4 <= n_chunks; ch += 4) {
+    a0 += pp[(size_t)ch * total + i];
+    a1 += pp[(size_t)(ch + 1) * total + i];
+    a2 += pp[(size_t)(ch + 2) * total + i];
+    a3 += pp[(size_t)(ch + 3) * total + i];
+  }
+  for (; ch < n_chunks; ++ch) a0 += pp[(size_t)ch * total + i];
+  p[i] = (a0 + a1) + (a2 + a3);
+}
+
+// Y[v][r] = act(W[r, :] . [Xa[v]; Xb[v]] + bias[r]) for every vector v < nv and output row
+// r < rows; the input of vector v is Xa[v] (na values) followed by Xb[v] (nb values, may be
+// 0).  W is row-major fp32 with na + nb <= 512 columns, na and nb multiples of 4.  Warp w of
+// CTA c takes row r = 8c + w: its W row stays in registers (lane: columns 4*lane + 128*k).
 template <bool kRelu>
-__device__ void gemv_rows(const float* __restrict__ W, const float* __restrict__ bias, const float* x, int rows,
-                          int cols, float* y) {
+__global__ void __launch_bounds__(kMlpThreads)
+mlp_layer_kernel(const float* __restrict__ Xa, int na, const float* __restrict__ Xb, int nb,
+                 const float* __restrict__ W, const float* __restrict__ bias, int rows, int nv,
+                 float* __restrict__ Y) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  for (int r = kGemvRows * warp; r < rows; r += kGemvRows * kMlpWarps) {
-    float s[kGemvRows];
+  const int r = blockIdx.x * kMlpWarps + warp;
+  if (r >= rows) return;
+  const int in = na + nb;
+  float4 w[4];
 #pragma unroll
-    for (int u = 0; u < kGemvRows; ++u) s[u] = 0.f;
-    for (int c = 4 * lane; c < cols; c += 128) {
-      const float4 xv = *reinterpret_cast<const float4*>(x + c);
-      float4 wv[kGemvRows];
+  for (int k = 0; k < 4; ++k) {
+    const int c = 4 * lane + 128 * k;
+    w[k] = c < in ? __ldg(reinterpret_cast<const float4*>(W + (size_t)r * in + c)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  const float br = bias[r];
+  for (int v = 0; v < nv; ++v) {
+    float s = 0.f;
 #pragma unroll
-      for (int u = 0; u < kGemvRows; ++u)
-        wv[u] = r + u < rows ? __ldg(reinterpret_cast<const float4*>(W + (size_t)(r + u) * cols + c))
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int u = 0; u < kGemvRows; ++u)
-        s[u] += wv[u].x * xv.x + wv[u].y * xv.y + wv[u].z * xv.z + wv[u].w * xv.w;
+    for (int k = 0; k < 4; ++k) {
+      const int c = 4 * lane + 128 * k;
+      if (c < in) {
+        const float4 x = c < na ? *reinterpret_cast<const float4*>(Xa + (size_t)v * na + c)
+                                : *reinterpret_cast<const float4*>(Xb + (size_t)v * nb + (c - na));
+        s += w[k].x * x.x + w[k].y * x.y + w[k].z * x.z + w[k].w * x.w;
+      }
     }
-#pragma unroll
-    for (int u = 0; u < kGemvRows; ++u) {
-      const float t = warp_sum(s[u]);
-      if (lane == 0 && r + u < rows) y[r + u] = kRelu ? fmaxf(t + bias[r + u], 0.f) : t + bias[r + u];
-    }
+    s = warp_sum(s);
+    if (lane == 0) Y[(size_t)v * rows + r] = kRelu ? fmaxf(s + br, 0.f) : s + br;
   }
 }
 
-// grid (H_kv, B): p = sum of the projection partials of head h, then the task MLP,
-// the router MLP on [p; tau], the head's output row and the threshold.
+// z[b][h] = w_o[h] . u[b*H_kv + h] + b_o[h]; head_mode = (z > 0).  One warp per (b, h).
 __global__ void __launch_bounds__(kMlpThreads)
-router_mlp_kernel(const float* __restrict__ pp, int n_chunks, int B, int H_kv, int d, ea_router_weights w,
-                  int32_t* __restrict__ head_mode, float* __restrict__ logits) {
-  extern __shared__ __align__(16) float sm[];
-  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const int N = H_kv * d;
-  float* p = sm;                  // [2d]: p then tau (the router MLP input [p; tau])
-  float* tau = p + d;
-  float* hid = p + 2 * d;         // [4d]
-  float* u = hid + 4 * d;         // [4d]
-  float* part = u + 4 * d;        // [kMlpThreads]
-  float* red = part + kMlpThreads;  // [kMlpWarps]
-  {
-    const int lanes = kMlpThreads / d, c = tid % d, cl = tid / d;
-    const float* src = pp + (size_t)b * N + (size_t)h * d + c;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    int ch = cl;
-    for (; ch + 7 * lanes < n_chunks; ch += 8 * lanes) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) acc[k] += src[(size_t)(ch + k * lanes) * B * N];
-    }
-    for (; ch < n_chunks; ch += lanes) acc[0] += src[(size_t)ch * B * N];
-    part[tid] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-  }
-  __syncthreads();
-  if (tid < d) {
-    float s = 0.f;
-    for (int l = 0; l < kMlpThreads / d; ++l) s += part[l * d + tid];
-    p[tid] = s;
-  }
-  __syncthreads();
-  gemv_rows<true>(w.w_t1, w.b_t1, p, 4 * d, d, hid);       // task MLP, hidden layer
-  __syncthreads();
-  gemv_rows<false>(w.w_t2, w.b_t2, hid, d, 4 * d, tau);    // task representation tau
-  __syncthreads();
-  gemv_rows<true>(w.w_r1, w.b_r1, p, 4 * d, 2 * d, u);     // router MLP on [p; tau]
-  __syncthreads();
+router_out_kernel(const float* __restrict__ u, int n4, int BH, int H_kv, const float* __restrict__ w_o,
+                  const float* __restrict__ b_o, int32_t* __restrict__ head_mode, float* __restrict__ logits) {
+  const int v = blockIdx.x * kMlpWarps + threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (v >= BH) return;
+  const int h = v % H_kv;
   float s = 0.f;
-  for (int j = tid; j < 4 * d; j += kMlpThreads) s += w.w_o[(size_t)h * 4 * d + j] * u[j];
+  for (int j = lane; j < n4; j += 32) s += w_o[(size_t)h * n4 + j] * u[(size_t)v * n4 + j];
   s = warp_sum(s);
-  if (tid % 32 == 0) red[tid / 32] = s;
-  __syncthreads();
-  if (tid == 0) {
-    float z = w.b_o[h];
-    for (int i = 0; i < kMlpWarps; ++i) z += red[i];
-    head_mode[b * H_kv + h] = z > 0.f ? 1 : 0;
-    if (logits) logits[b * H_kv + h] = z;
+  if (lane == 0) {
+    const float z = s + b_o[h];
+    head_mode[v] = z > 0.f ? 1 : 0;
+    if (logits) logits[v] = z;
   }
 }
 
@@ -317,16 +308,18 @@ PoolPlan plan_pool(int B, int S, int D, int n_boundary, int vec) {
 
 static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Workspace: pooling partial sums [n_splits][B][D], then projection partials
-// [ceil(D/64)][B][H_kv*d].
+// Workspace: pooling partial sums [n_splits][B][D], projection partials
+// [ceil(D/32)][B][H_kv*d], then the MLP vectors p [B*H_kv][d], hid [.][4d], tau [.][d],
+// u [.][4d].
 static size_t partial_bytes(int B, int S, int D, int n_boundary) {
   PoolPlan pl4 = plan_pool(B, S, D, n_boundary, 4), pl8 = plan_pool(B, S, D, n_boundary, 8);
   return align256((size_t)max(pl4.n_splits, pl8.n_splits) * B * D * sizeof(float));
 }
 static size_t proj_bytes(int B, int D, int N) { return align256((size_t)cdiv(D, kProjRows) * B * N * sizeof(float)); }
+static size_t mlp_bytes(int B, int N) { return align256((size_t)B * N * 10 * sizeof(float)); }
 
 size_t router_workspace_bytes(int B, int S, int D, int H_kv, int d, int n_boundary) {
-  return partial_bytes(B, S, D, n_boundary) + proj_bytes(B, D, H_kv * d);
+  return partial_bytes(B, S, D, n_boundary) + proj_bytes(B, D, H_kv * d) + mlp_bytes(B, H_kv * d);
 }
 
 ea_status launch_router(const void* hidden, ea_dtype dtype, int B, int S, int D, int H_kv, int d,
@@ -349,8 +342,21 @@ ea_status launch_router(const void* hidden, ea_dtype dtype, int B, int S, int D,
     project_kernel<float><<<n_chunks, kProjThreads, 0, st>>>(
         partial, pl.n_splits, B, D, 1.0f / (float)pl.n_rows, static_cast<const float*>(w->w_k), N, pp);
   }
-  const size_t smem = sizeof(float) * ((size_t)10 * d + kMlpThreads + kMlpWarps);
-  router_mlp_kernel<<<dim3(H_kv, B), kMlpThreads, smem, st>>>(pp, n_chunks, B, H_kv, d, *w, head_mode, logits);
+  if (cudaGetLastError() != cudaSuccess) return EA_ERR_CUDA;
+  float* p = reinterpret_cast<float*>(reinterpret_cast<char*>(pp) + proj_bytes(B, D, N));
+  const int BH = B * H_kv;
+  float* hid = p + (size_t)BH * d;
+  float* tau = hid + (size_t)BH * 4 * d;
+  float* u = tau + (size_t)BH * d;
+  proj_reduce_kernel<<<cdiv(B * N, 256), 256, 0, st>>>(pp, n_chunks, B * N, p);
+  mlp_layer_kernel<true><<<cdiv(4 * d, kMlpWarps), kMlpThreads, 0, st>>>(p, d, nullptr, 0, w->w_t1, w->b_t1, 4 * d,
+                                                                        BH, hid);      // task MLP, hidden layer
+  mlp_layer_kernel<false><<<cdiv(d, kMlpWarps), kMlpThreads, 0, st>>>(hid, 4 * d, nullptr, 0, w->w_t2, w->b_t2, d,
+                                                                      BH, tau);        // task representation
+  mlp_layer_kernel<true><<<cdiv(4 * d, kMlpWarps), kMlpThreads, 0, st>>>(p, d, tau, d, w->w_r1, w->b_r1, 4 * d,
+                                                                        BH, u);        // router MLP on [p; tau]
+  router_out_kernel<<<cdiv(BH, kMlpWarps), kMlpThreads, 0, st>>>(u, 4 * d, BH, H_kv, w->w_o, w->b_o, head_mode,
+                                                                 logits);
   return cudaGetLastError() == cudaSuccess ? EA_OK : EA_ERR_CUDA;
 }
 
