@@ -146,6 +146,8 @@ WORKLOADS = {w.name: w for w in [
     _w("llama3-8b-s32k-stack8", 1, 32768, 4096, 32, 8, 128, "bf16", 128, 2048, (STREAMING,) * 8,
        ("fixed", 4), layers=8, needle=(16384, 16448), omega_static=0.5,
        note="8 layers; k = floor(0.5 * 8 * 8) = 32 KV heads keep full attention, 32 stream"),
+    _w("small-stack3-s1000", 1, 1000, 256, 8, 2, 128, "bf16", 64, 300, (STREAMING,) * 2, ("fixed", 1),
+       layers=3, needle=(400, 432), omega_static=0.5, note="3 small layers with static assignment"),
     _w("small-xattn-g4-s2560", 2, 2560, 256, 8, 2, 128, "bf16", 64, 300, (BLOCK_SPARSE,) * 2,
        ("per_sample", (1, 2)), pos_amp=1.5, **_XA),
     _w("small-xattn-g7-s1000", 1, 1000, 384, 14, 2, 128, "bf16", 0, 1, (BLOCK_SPARSE,) * 2,
