@@ -189,8 +189,9 @@ def run_cuda(args):
     o = torch.empty_like(q)
     xattn = w.layout == "xattn"
     if xattn:
-        pat = abi.Pattern.for_xattn(w.B, w.S, w.H_kv, w.n_sink, w.window, w.kind_if_dense, w.kind_if_sparse)
-        xws = torch.zeros(abi.ea_xattn_workspace_size(w.B, w.S, w.H_q, w.H_kv, w.stride), dtype=torch.uint8,
+        pat = abi.Pattern.for_xattn(w.B, w.S, w.H_kv, w.n_sink, w.window, w.kind_if_dense, w.kind_if_sparse,
+                                    block=w.block)
+        xws = torch.zeros(abi.ea_xattn_workspace_size(w.B, w.S, w.H_q, w.H_kv, w.stride, w.block), dtype=torch.uint8,
                           device=dev)
     else:
         pat = abi.Pattern.from_workloads(inp["pattern"])
@@ -767,7 +768,7 @@ def oracle_sample(w, inp, budget_s):
               kind_if_dense=pat.kind_if_dense, kind_if_sparse=pat.kind_if_sparse)
     k64, v64 = f64(inp["k"]), f64(inp["v"])
     xattn = w.layout == "xattn"
-    n_qb = -(-w.S // 128)
+    n_qb = -(-w.S // w.block)
     bs_heads = [(b, h) for b in range(w.B) for h in range(w.H_kv)
                 if (w.kind_if_sparse[h] if mode[b, h] else w.kind_if_dense[h]) == wl.BLOCK_SPARSE]
     sel = {}                                  # (b, h, qb) -> kept key blocks (oracle selection)
@@ -777,12 +778,12 @@ def oracle_sample(w, inp, budget_s):
         nonlocal t_sel
         t1 = time.perf_counter()
         for qb in qbs:
-            lo, hi = qb * 128, min((qb + 1) * 128, w.S)
+            lo, hi = qb * w.block, min((qb + 1) * w.block, w.S)
             for b, h in bs_heads:
                 if (b, h, qb) in sel:
                     continue
                 a = oracle.xattention.row_importance(f64(inp["q"][b:b + 1, lo:hi]), k64[b:b + 1, :hi], 0, h, qb,
-                                                     w.stride, 128, q_first_row=lo)
+                                                     w.stride, w.block, q_first_row=lo)
                 sel[(b, h, qb)] = oracle.xattention.select_blocks(a, qb, w.tau)
         t_sel += time.perf_counter() - t1
 
@@ -800,7 +801,7 @@ def oracle_sample(w, inp, budget_s):
         rows = np.unique(np.linspace(0, w.S - 1, n_rows).astype(np.int64) + rows_done % 7)
         rows = rows[rows < w.S]
         if xattn:
-            select_rows(np.unique(rows // 128))
+            select_rows(np.unique(rows // w.block))
             pd["row_ptr"], pd["cols"] = layout()
         t1 = time.perf_counter()
         oracle.attention.hybrid_attention_rows(f64(inp["q"][:, rows]), k64, v64, mode, pd, rows, q_row_index=rows)

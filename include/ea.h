@@ -200,7 +200,7 @@ EA_API ea_status ea_attn_scheduled(const void* q, const void* k, const void* v, 
  *   R[i, j]   = sum_{m<st} q[i*st+m] . k[j*st+st-1-m]       (reduced i, j < S/st)
  *   P[i, :]   = softmax over j <= i of R[i, j] * scale / st  (scale as below)
  *   A[qb, kb] = mean over the G query heads of KV head h of the P mass of the
- *               128 x 128 tile (qb, kb)
+ *               block x block tile (qb, kb), block = pattern->block (64 or 128)
  *   row qb    = {qb} plus blocks in descending A (ties: lower index) while the
  *               kept mass < tau * sum_kb A[qb, kb]
  * Rows are computed for every (b, h) whose kind under head_mode is
@@ -209,17 +209,18 @@ EA_API ea_status ea_attn_scheduled(const void* q, const void* k, const void* v, 
  * `stream` with no host round trip.
  * ---------------------------------------------------------------------- */
 
-/* Bytes of workspace ea_xattn_block_select needs: per reduced row (S/stride of
- * them per query head) one float per 128-key block and per 128-row reduced
- * tile, plus O(B*H_kv*S/128) for the counts and bitmaps. */
-EA_API size_t ea_xattn_workspace_size(int B, int S, int H_q, int H_kv, int stride);
+/* Bytes of workspace ea_xattn_block_select needs for layouts at block edge
+ * `block` (64 or 128): per reduced row (S/stride of them per query head) one
+ * float per key block and per 128-row reduced tile, plus O(B*H_kv*S/block)
+ * for the counts and bitmaps. */
+EA_API size_t ea_xattn_workspace_size(int B, int S, int H_q, int H_kv, int stride, int block);
 
 /* q: device [B, S, H_q, 128] bf16, k: device [B, S, H_kv, 128] bf16 (16-byte
- * aligned).  stride in {4, 8, 16} with S % stride == 0; S <= 262144;
- * (H_q / H_kv) * 128 / stride <= 1024; 0 <= tau <= 1.  pattern: kinds,
- * block == 128 and softmax_scale are read; its bs_* fields are ignored.
- * row_ptr: device int32 [B*H_kv*ceil(S/128) + 1] (written).  cols: device int32
- * with cols_capacity >= B*H_kv*n_qb*(n_qb+1)/2 entries, n_qb = ceil(S/128)
+ * aligned).  stride in {4, 8, 16} with S % stride == 0; ceil(S/block) <= 2048;
+ * (H_q / H_kv) * block / stride <= 1024; 0 <= tau <= 1.  pattern: kinds,
+ * block (64 or 128) and softmax_scale are read; its bs_* fields are ignored.
+ * row_ptr: device int32 [B*H_kv*n_qb + 1] (written), n_qb = ceil(S/block).
+ * cols: device int32 with cols_capacity >= B*H_kv*n_qb*(n_qb+1)/2 entries
  * (the first row_ptr[last] are written, ascending within each row).
  * block_scores: NULL, or device float [B, H_kv, n_qb, n_qb] receiving A (zero
  * above the diagonal and on rows of other kinds).  Buffers are the caller's;

@@ -94,7 +94,7 @@ def _lib():
                                                  POINTER(RouterWeights), POINTER(RouterParams), c_void_p,
                                                  c_void_p, c_void_p]
         lib.ea_xattn_workspace_size.restype = c_size_t
-        lib.ea_xattn_workspace_size.argtypes = [c_int, c_int, c_int, c_int, c_int]
+        lib.ea_xattn_workspace_size.argtypes = [c_int, c_int, c_int, c_int, c_int, c_int]
         lib.ea_xattn_block_select.restype = st
         lib.ea_xattn_block_select.argtypes = [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p,
                                               POINTER(PatternParams), c_int, c_float, c_void_p, c_void_p,
@@ -166,12 +166,12 @@ class Pattern:
 
     @classmethod
     def for_xattn(cls, B, S, H_kv, n_sink, window, kind_if_dense, kind_if_sparse, softmax_scale=0.0,
-                  device="cuda"):
+                  device="cuda", block=128):
         """A pattern whose block layout ea_xattn_block_select fills: row_ptr and cols are
         device buffers of the sizes that call needs (cols at its worst-case capacity)."""
-        n_qb = -(-S // 128)
-        return cls(n_sink, window, 128, np.zeros(B * H_kv * n_qb + 1, np.int32),
-                   np.zeros(xattn_cols_capacity(B, S, H_kv), np.int32), kind_if_dense, kind_if_sparse,
+        n_qb = -(-S // block)
+        return cls(n_sink, window, block, np.zeros(B * H_kv * n_qb + 1, np.int32),
+                   np.zeros(xattn_cols_capacity(B, S, H_kv, block), np.int32), kind_if_dense, kind_if_sparse,
                    softmax_scale, device)
 
     @classmethod
@@ -280,14 +280,14 @@ def ea_attn_scheduled(q, k, v, head_mode, pattern: Pattern, o, workspace, stream
     _check(_lib().ea_attn_scheduled(*args), "ea_attn_scheduled")
 
 
-def xattn_cols_capacity(B: int, S: int, H_kv: int) -> int:
+def xattn_cols_capacity(B: int, S: int, H_kv: int, block: int = 128) -> int:
     """Entries ea_xattn_block_select may write into cols: every causal block of every row."""
-    n_qb = -(-S // 128)
+    n_qb = -(-S // block)
     return B * H_kv * n_qb * (n_qb + 1) // 2
 
 
-def ea_xattn_workspace_size(B: int, S: int, H_q: int, H_kv: int, stride: int = 8) -> int:
-    return int(_lib().ea_xattn_workspace_size(B, S, H_q, H_kv, stride))
+def ea_xattn_workspace_size(B: int, S: int, H_q: int, H_kv: int, stride: int = 8, block: int = 128) -> int:
+    return int(_lib().ea_xattn_workspace_size(B, S, H_q, H_kv, stride, block))
 
 
 def ea_xattn_block_select(q, k, head_mode, pattern: Pattern, workspace, stride: int = 8, tau: float = 0.9,

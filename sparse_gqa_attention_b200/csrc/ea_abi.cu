@@ -252,10 +252,10 @@ ea_status ea_static_head_assignment(const float* scores, int L, int B, int H_q, 
   return launch_assignment(scores, L, B, H_q, H_kv, k_full, head_mode, as_stream(stream));
 }
 
-size_t ea_xattn_workspace_size(int B, int S, int H_q, int H_kv, int stride) {
+size_t ea_xattn_workspace_size(int B, int S, int H_q, int H_kv, int stride, int block) {
   if (B < 1 || S < 1 || H_q < 1 || H_kv < 1 || H_q % H_kv != 0) return 0;
-  if (!xattn_shape_ok(S, H_q, H_kv, stride)) return 0;
-  return xattn_workspace_bytes(B, S, H_q, H_kv, stride);
+  if (!xattn_shape_ok(S, H_q, H_kv, stride, block)) return 0;
+  return xattn_workspace_bytes(B, S, H_q, H_kv, stride, block);
 }
 
 ea_status ea_xattn_block_select(const void* q, const void* k, ea_dtype dtype, int B, int S, int H_q, int H_kv, int d,
@@ -274,11 +274,12 @@ ea_status ea_xattn_block_select(const void* q, const void* k, ea_dtype dtype, in
   pp.bs_nnz = cols_capacity;
   PatternDev pd;
   if (ea_status s = check_pattern(head_mode, &pp, B, S, S, 0, H_q, H_kv, d, &pd)) return s;
-  if (pp.block != kTile) return EA_ERR_UNSUPPORTED;
-  if (!xattn_shape_ok(S, H_q, H_kv, stride)) return EA_ERR_UNSUPPORTED;
-  const long long n_qb = cdiv(S, kTile);
+  if (!xattn_shape_ok(S, H_q, H_kv, stride, pp.block)) return EA_ERR_UNSUPPORTED;
+  pd.n_qb = cdiv(S, pp.block);   // the layout is written at the pattern's block edge
+  const long long n_qb = pd.n_qb;
   if (cols_capacity < (long long)B * H_kv * n_qb * (n_qb + 1) / 2) return EA_ERR_INVALID_ARG;
-  if (ea_status s = check_ws(workspace, workspace_bytes, xattn_workspace_bytes(B, S, H_q, H_kv, stride))) return s;
+  if (ea_status s = check_ws(workspace, workspace_bytes, xattn_workspace_bytes(B, S, H_q, H_kv, stride, pp.block)))
+    return s;
   return launch_xattn(q, k, head_mode, pd, B, S, H_q, H_kv, stride, tau, row_ptr, cols, block_scores, workspace,
                       as_stream(stream));
 }

@@ -33,8 +33,8 @@ ea_status launch_attn_tc64(const void* q, const void* k, const void* v, void* o,
                            cudaStream_t st);
 
 // XAttention block selection (ea_xattn.cu).
-bool xattn_shape_ok(int S, int H_q, int H_kv, int stride);
-size_t xattn_workspace_bytes(int B, int S, int H_q, int H_kv, int stride);
+bool xattn_shape_ok(int S, int H_q, int H_kv, int stride, int block);
+size_t xattn_workspace_bytes(int B, int S, int H_q, int H_kv, int stride, int block);
 ea_status launch_xattn(const void* q, const void* k, const int32_t* head_mode, const PatternDev& pd, int B, int S,
                        int H_q, int H_kv, int stride, float tau, int32_t* row_ptr, int32_t* cols, float* scores,
                        void* workspace, cudaStream_t st);

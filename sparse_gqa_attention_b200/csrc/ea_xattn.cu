@@ -71,18 +71,19 @@ struct XLayout {
   size_t plan, m_part, s_part, counts, bitmap, total;
 };
 size_t up256(size_t x) { return (x + 255) / 256 * 256; }
-XLayout x_layout(int B, int S, int H_q, int H_kv, int st) {
+// blk: the layout's block edge (64 or 128); a 128-column reduced tile holds 128*st/blk blocks.
+XLayout x_layout(int B, int S, int H_q, int H_kv, int st, int blk) {
   XLayout L;
   L.n_red = S / st;
   L.n_rt = cdiv(L.n_red, XT);
-  L.n_qb = cdiv(S, kTile);
+  L.n_qb = cdiv(S, blk);
   L.words = cdiv(L.n_qb, 32);
   const size_t rows_red = (size_t)B * H_q * L.n_red;
   const size_t n_rows = (size_t)B * H_kv * L.n_qb;
   L.plan = kXsHeader;
   L.m_part = L.plan + up256((size_t)B * H_q * 4);
   L.s_part = L.m_part + up256(rows_red * L.n_rt * 4);
-  L.counts = L.s_part + up256(rows_red * L.n_rt * st * 4);
+  L.counts = L.s_part + up256(rows_red * L.n_rt * (XT * st / blk) * 4);
   L.bitmap = L.counts + up256(n_rows * 4);
   L.total = L.bitmap + up256(n_rows * L.words * 4);
   return L;
@@ -170,18 +171,19 @@ __global__ void xattn_plan_kernel(const int32_t* __restrict__ head_mode, Pattern
   if (bad) atomicOr(hdr + kWsStatus / 4, bad);
 }
 
-// Partial softmax sums of one reduced row over one 128-column tile: sg[g] = sum of
-// exp2(x*sl2 - ms) over the live columns of block g, ms = sl2 * (max over live columns).
-template <int ST, bool kDiag>
-__device__ __forceinline__ float x_row_tile(const float (&x)[XT], int lim, float sl2, float (&sg)[ST]) {
-  constexpr int BW = XT / ST;
+// Partial softmax sums of one reduced row over one 128-column tile holding NB blocks:
+// sg[g] = sum of exp2(x*sl2 - ms) over the live columns of block g, ms = sl2 * (max over
+// live columns).
+template <int NB, bool kDiag>
+__device__ __forceinline__ float x_row_tile(const float (&x)[XT], int lim, float sl2, float (&sg)[NB]) {
+  constexpr int BW = XT / NB;
   float mx = -INFINITY;
 #pragma unroll
   for (int e = 0; e < XT; ++e)
     if (!kDiag || e <= lim) mx = fmaxf(mx, x[e]);
   const float ms = mx * sl2;
 #pragma unroll
-  for (int g = 0; g < ST; ++g) {
+  for (int g = 0; g < NB; ++g) {
     float a0 = 0.f, a1 = 0.f;
 #pragma unroll
     for (int e = 0; e < BW; e += 2) {
@@ -194,7 +196,8 @@ __device__ __forceinline__ float x_row_tile(const float (&x)[XT], int lim, float
   return ms;
 }
 
-template <int ST>
+// ST: antidiagonal stride; NB: blocks per 128-column reduced tile (ST at block 128, 2*ST at 64).
+template <int ST, int NB>
 __global__ void __launch_bounds__(kXThreads, 1)
 xattn_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, int H_q,
                    int H_kv, int n_red, int n_rt, float sl2, const int* __restrict__ plan,
@@ -295,7 +298,7 @@ xattn_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int wq = warp % 4;
     const int row = wq * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(wq * 32) << 16);
-    const int pitch = n_rt * ST;
+    const int pitch = n_rt * NB;
     int tile = 0;
     bool ok = true;
     for (int it = 0; ok; ++it) {
@@ -328,12 +331,12 @@ xattn_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_arrive(c.bar(X_AEMPTY + a));
           }
           if (i < n_red && ct <= I.r) {
-            float sg[ST];
+            float sg[NB];
             const float ms =
-                ct < I.r ? x_row_tile<ST, false>(x, XT - 1, sl2, sg) : x_row_tile<ST, true>(x, row, sl2, sg);
-            float* sp = s_part + rrow * pitch + ct * ST;
+                ct < I.r ? x_row_tile<NB, false>(x, XT - 1, sl2, sg) : x_row_tile<NB, true>(x, row, sl2, sg);
+            float* sp = s_part + rrow * pitch + ct * NB;
 #pragma unroll
-            for (int g = 0; g < ST; g += 4)
+            for (int g = 0; g < NB; g += 4)
               *reinterpret_cast<float4*>(sp + g) = make_float4(sg[g], sg[g + 1], sg[g + 2], sg[g + 3]);
             m_part[rrow * n_rt + ct] = ms;
           }
@@ -352,12 +355,12 @@ xattn_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 }
 
 // One CTA per (query block qb, KV head h, sample b).
-template <int ST>
+template <int ST, int NB>
 __global__ void __launch_bounds__(kSelThreads)
 xattn_select_kernel(const int32_t* __restrict__ head_mode, PatternDev p, int H_q, int H_kv, int n_red, int n_rt,
                     float tau, const float* __restrict__ m_part, const float* __restrict__ s_part,
                     uint32_t* __restrict__ counts, uint32_t* __restrict__ bitmap, float* __restrict__ scores) {
-  constexpr int BW = XT / ST;                  // reduced rows per 128-row block
+  constexpr int BW = XT / NB;                  // reduced rows (and columns) per block
   __shared__ float a[kMaxQb];
   __shared__ unsigned long long keys[kMaxQb];
   __shared__ float rowM[kMaxSelRows], rowInvL[kMaxSelRows];
@@ -378,7 +381,7 @@ xattn_select_kernel(const int32_t* __restrict__ head_mode, PatternDev p, int H_q
   }
   const int G = H_q / H_kv;
   const int i0 = qb * BW, nr = min(BW, n_red - i0), rows = G * nr;
-  const int pitch = n_rt * ST;
+  const int pitch = n_rt * NB;
 
   // Row maxima M (log2 units) and 1 / row sums, one warp per reduced row.
   for (int rr = warp; rr < rows; rr += kSelThreads / 32) {
@@ -392,7 +395,7 @@ xattn_select_kernel(const int32_t* __restrict__ head_mode, PatternDev p, int H_q
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float L = 0.f;
-    for (int kb = lane; kb < n_t * ST; kb += 32) L += srow[kb] * ex2(mrow[kb / ST] - M);
+    for (int kb = lane; kb < n_t * NB; kb += 32) L += srow[kb] * ex2(mrow[kb / NB] - M);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
     if (lane == 0) {
@@ -410,7 +413,7 @@ xattn_select_kernel(const int32_t* __restrict__ head_mode, PatternDev p, int H_q
     for (int rr = 0; rr < rows; ++rr) {
       const int g = rr / nr, i = i0 + rr % nr;
       const size_t rrow = ((size_t)b * H_q + h * G + g) * n_red + i;
-      acc += s_part[rrow * pitch + kb] * ex2(m_part[rrow * n_rt + kb / ST] - rowM[rr]) * rowInvL[rr];
+      acc += s_part[rrow * pitch + kb] * ex2(m_part[rrow * n_rt + kb / NB] - rowM[rr]) * rowInvL[rr];
     }
     a[kb] = acc * inv_g;
     if (scores) scores[row * n_qb + kb] = acc * inv_g;
@@ -609,11 +612,11 @@ int x_sm_count() {
   return n;
 }
 
-template <int ST>
+template <int ST, int NB>
 ea_status launch_st(const void* q, const void* k, const int32_t* head_mode, const PatternDev& pd, int B, int S,
                     int H_q, int H_kv, float tau, int32_t* row_ptr, int32_t* cols, float* scores, void* workspace,
                     cudaStream_t st) {
-  const XLayout L = x_layout(B, S, H_q, H_kv, ST);
+  const XLayout L = x_layout(B, S, H_q, H_kv, ST, XT * ST / NB);
   CUtensorMap mq, mk;
   if (!make_map5(&mq, q, B, S, H_q, ST, XT) || !make_map5(&mk, k, B, S, H_kv, ST, XN)) return EA_ERR_CUDA;
   char* ws = static_cast<char*>(workspace);
@@ -627,7 +630,7 @@ ea_status launch_st(const void* q, const void* k, const int32_t* head_mode, cons
 
   xattn_plan_kernel<<<1, 32, 0, st>>>(head_mode, pd, B, H_q, H_kv, hdr, plan);
   if (cudaGetLastError() != cudaSuccess) return EA_ERR_CUDA;
-  auto kern = xattn_score_kernel<ST>;
+  auto kern = xattn_score_kernel<ST, NB>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kXSmemBytes) != cudaSuccess)
     return EA_ERR_CUDA;
   const long long max_work = (long long)B * H_q * L.n_rt;
@@ -635,7 +638,7 @@ ea_status launch_st(const void* q, const void* k, const int32_t* head_mode, cons
   kern<<<grid, kXThreads, kXSmemBytes, st>>>(mq, mk, H_q, H_kv, L.n_red, L.n_rt, sl2, plan, hdr, m_part, s_part);
   if (cudaGetLastError() != cudaSuccess) return EA_ERR_CUDA;
   dim3 sgrid(L.n_qb, H_kv, B);
-  xattn_select_kernel<ST><<<sgrid, kSelThreads, 0, st>>>(head_mode, pd, H_q, H_kv, L.n_red, L.n_rt, tau, m_part,
+  xattn_select_kernel<ST, NB><<<sgrid, kSelThreads, 0, st>>>(head_mode, pd, H_q, H_kv, L.n_red, L.n_rt, tau, m_part,
                                                          s_part, counts, bitmap, scores);
   if (cudaGetLastError() != cudaSuccess) return EA_ERR_CUDA;
   const int n_rows = B * H_kv * L.n_qb;
@@ -647,25 +650,34 @@ ea_status launch_st(const void* q, const void* k, const int32_t* head_mode, cons
 
 }  // namespace
 
-bool xattn_shape_ok(int S, int H_q, int H_kv, int stride) {
+bool xattn_shape_ok(int S, int H_q, int H_kv, int stride, int block) {
   if (stride != 4 && stride != 8 && stride != 16) return false;
-  if (S % stride != 0 || cdiv(S, kTile) > kMaxQb) return false;
-  return (long long)(H_q / H_kv) * (kTile / stride) <= kMaxSelRows;
+  if (block != 64 && block != kTile) return false;
+  if (S % stride != 0 || cdiv(S, block) > kMaxQb) return false;
+  return (long long)(H_q / H_kv) * (block / stride) <= kMaxSelRows;
 }
 
-size_t xattn_workspace_bytes(int B, int S, int H_q, int H_kv, int stride) {
-  return x_layout(B, S, H_q, H_kv, stride).total;
+size_t xattn_workspace_bytes(int B, int S, int H_q, int H_kv, int stride, int block) {
+  return x_layout(B, S, H_q, H_kv, stride, block).total;
 }
 
 ea_status launch_xattn(const void* q, const void* k, const int32_t* head_mode, const PatternDev& pd, int B, int S,
                        int H_q, int H_kv, int stride, float tau, int32_t* row_ptr, int32_t* cols, float* scores,
                        void* workspace, cudaStream_t st) {
+  const bool b64 = pd.block == 64;
+#define EA_XATTN_CASE(STRIDE)                                                                                  \
+  case STRIDE:                                                                                                 \
+    return b64 ? launch_st<STRIDE, 2 * STRIDE>(q, k, head_mode, pd, B, S, H_q, H_kv, tau, row_ptr, cols, scores, \
+                                               workspace, st)                                                  \
+               : launch_st<STRIDE, STRIDE>(q, k, head_mode, pd, B, S, H_q, H_kv, tau, row_ptr, cols, scores,   \
+                                           workspace, st);
   switch (stride) {
-    case 4: return launch_st<4>(q, k, head_mode, pd, B, S, H_q, H_kv, tau, row_ptr, cols, scores, workspace, st);
-    case 8: return launch_st<8>(q, k, head_mode, pd, B, S, H_q, H_kv, tau, row_ptr, cols, scores, workspace, st);
-    case 16: return launch_st<16>(q, k, head_mode, pd, B, S, H_q, H_kv, tau, row_ptr, cols, scores, workspace, st);
+    EA_XATTN_CASE(4)
+    EA_XATTN_CASE(8)
+    EA_XATTN_CASE(16)
     default: return EA_ERR_UNSUPPORTED;
   }
+#undef EA_XATTN_CASE
 }
 
 }  // namespace ea

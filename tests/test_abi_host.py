@@ -117,7 +117,7 @@ def _xattn_call(lib, S=1024, H_q=8, H_kv=2, d=128, dtype=None, stride=8, tau=0.9
     (dict(tau=-0.1), abi.EA_ERR_INVALID_ARG),
     (dict(dtype=abi.EA_DT_F32), abi.EA_ERR_UNSUPPORTED),
     (dict(d=64), abi.EA_ERR_UNSUPPORTED),
-    (dict(block=64), abi.EA_ERR_UNSUPPORTED),
+    (dict(block=32), abi.EA_ERR_UNSUPPORTED),
     (dict(cap=10), abi.EA_ERR_INVALID_ARG),
     (dict(ws_bytes=1024), abi.EA_ERR_INVALID_ARG),
     (dict(H_q=7), abi.EA_ERR_INVALID_ARG),
@@ -130,13 +130,19 @@ def test_xattn_argument_checks(lib, case, expect):
 def test_xattn_workspace_size(lib):
     B, S, H_q, H_kv, st = 1, 65536, 28, 4, 8
     n_red, n_rt, n_qb = S // st, S // st // 128, S // 128
-    n = abi.ea_xattn_workspace_size(B, S, H_q, H_kv, st)
+    n = abi.ea_xattn_workspace_size(B, S, H_q, H_kv, st, 128)
     parts = B * H_q * n_red * n_rt * 4 * (1 + st)          # tile maxima + per-block partial sums
     assert parts < n < parts + 1024 + B * H_kv * n_qb * 4 * (1 + n_qb // 32 + 1) + 1024
     assert n % 256 == 0
-    assert abi.ea_xattn_workspace_size(B, S, H_q, H_kv, 6) == 0
-    assert abi.ea_xattn_workspace_size(B, 1001, H_q, H_kv, 8) == 0
+    assert abi.ea_xattn_workspace_size(B, S, H_q, H_kv, 6, 128) == 0
+    assert abi.ea_xattn_workspace_size(B, 1001, H_q, H_kv, 8, 128) == 0
+    assert abi.ea_xattn_workspace_size(B, S, H_q, H_kv, 8, 96) == 0
+    # block 64: twice the per-block partial sums of block 128
+    n64 = abi.ea_xattn_workspace_size(B, S, H_q, H_kv, st, 64)
+    assert n64 > n + B * H_q * n_red * n_rt * 4 * st - 4096
+    assert abi.ea_xattn_workspace_size(1, 262144, 8, 8, 8, 64) == 0      # 4096 blocks of 64
     assert abi.xattn_cols_capacity(2, 300, 3) == 2 * 3 * 3 * 4 // 2
+    assert abi.xattn_cols_capacity(1, 300, 1, 64) == 5 * 6 // 2
 
 
 @pytest.mark.parametrize("case,expect", [

@@ -21,7 +21,7 @@ from tests import _gpu
 pytestmark = pytest.mark.gpu
 
 SMALL = ["small-xattn-g4-s2560", "small-xattn-g7-s1000", "small-xassa-g4-s1536"]
-FULL_SIZE = ["qwen-g7-s64k-xattn", "llama3-8b-s32k-xassa"]
+FULL_SIZE = ["qwen-g7-s64k-xattn", "llama3-8b-s32k-xassa", "qwen-g7-s64k-xattn-b64"]
 SEL_TOL = 1e-4
 
 
@@ -34,9 +34,11 @@ def run_xattn(w, q, k, head_mode, stride=None, tau=None, scores=True):
     ta = w.tau if tau is None else tau
     dq, dk = _gpu.to_dev(q, w.dtype), _gpu.to_dev(k, w.dtype)
     hm = torch.from_numpy(np.ascontiguousarray(head_mode, np.int32)).cuda()
-    pat = abi.Pattern.for_xattn(w.B, w.S, w.H_kv, w.n_sink, w.window, w.kind_if_dense, w.kind_if_sparse)
-    ws = torch.zeros(abi.ea_xattn_workspace_size(w.B, w.S, w.H_q, w.H_kv, st), dtype=torch.uint8, device="cuda")
-    n_qb = -(-w.S // 128)
+    pat = abi.Pattern.for_xattn(w.B, w.S, w.H_kv, w.n_sink, w.window, w.kind_if_dense, w.kind_if_sparse,
+                                block=w.block)
+    ws = torch.zeros(abi.ea_xattn_workspace_size(w.B, w.S, w.H_q, w.H_kv, st, w.block), dtype=torch.uint8,
+                     device="cuda")
+    n_qb = -(-w.S // w.block)
     sc = torch.full((w.B, w.H_kv, n_qb, n_qb), float("nan"), device="cuda") if scores else None
     abi.ea_xattn_block_select(dq, dk, hm, pat, ws, st, ta, sc)
     torch.cuda.synchronize()
@@ -71,7 +73,7 @@ def check_row(got, a, qb, tau):
 
 
 def check_layout_shape(w, mode, rp, cols):
-    n_qb = -(-w.S // 128)
+    n_qb = -(-w.S // w.block)
     assert rp[0] == 0 and np.all(np.diff(rp) >= 0)
     for b in range(w.B):
         for h in range(w.H_kv):
@@ -84,24 +86,30 @@ def check_layout_shape(w, mode, rp, cols):
                     assert len(row) == 0
 
 
-@pytest.mark.parametrize("name", SMALL)
-def test_small_scores_and_selection(name):
+def _w(name, block=128):
+    import dataclasses
     w = wl.WORKLOADS[name]
+    return w if block == w.block else dataclasses.replace(w, block=block)
+
+
+@pytest.mark.parametrize("name,block", [(n, 128) for n in SMALL] + [(n, 64) for n in SMALL])
+def test_small_scores_and_selection(name, block):
+    w = _w(name, block)
     q, k, v, _, _ = _gpu.cached_inputs(name)
     mode = _mode(w)
     rp, cols, sc, status, _ = run_xattn(w, q, k, mode)
     assert status == abi.EA_OK
     check_layout_shape(w, mode, rp, cols)
     qf, kf = _gpu.to_f64(q), _gpu.to_f64(k)
-    n_qb = -(-w.S // 128)
+    n_qb = -(-w.S // w.block)
     exact = total = 0
     for b in range(w.B):
         for h in range(w.H_kv):
             if _kinds(w, mode, b, h) != wl.BLOCK_SPARSE:
                 assert np.all(sc[b, h] == 0)
                 continue
-            A = ox.group_importance(qf, kf, b, h, w.stride, 128)
-            np.testing.assert_allclose(sc[b, h], A, rtol=1e-3, atol=2e-5 * 128 / w.stride)
+            A = ox.group_importance(qf, kf, b, h, w.stride, w.block)
+            np.testing.assert_allclose(sc[b, h], A, rtol=1e-3, atol=2e-5 * w.block / w.stride)
             for qb in range(n_qb):
                 r = (b * w.H_kv + h) * n_qb + qb
                 exact += check_row(cols[rp[r]:rp[r + 1]], A[qb], qb, w.tau)
@@ -117,13 +125,13 @@ def test_other_strides(stride):
     rp, cols, sc, status, _ = run_xattn(w, q, k, mode, stride=stride)
     assert status == abi.EA_OK
     qf, kf = _gpu.to_f64(q), _gpu.to_f64(k)
-    n_qb = -(-w.S // 128)
+    n_qb = -(-w.S // w.block)
     for b in range(w.B):
         for h in range(w.H_kv):
             if _kinds(w, mode, b, h) != wl.BLOCK_SPARSE:
                 continue
-            A = ox.group_importance(qf, kf, b, h, stride, 128)
-            np.testing.assert_allclose(sc[b, h], A, rtol=1e-3, atol=2e-5 * 128 / stride)
+            A = ox.group_importance(qf, kf, b, h, stride, w.block)
+            np.testing.assert_allclose(sc[b, h], A, rtol=1e-3, atol=2e-5 * w.block / stride)
             for qb in range(n_qb):
                 r = (b * w.H_kv + h) * n_qb + qb
                 check_row(cols[rp[r]:rp[r + 1]], A[qb], qb, w.tau)
@@ -135,7 +143,7 @@ def test_tau_zero_keeps_only_the_diagonal():
     mode = _mode(w)
     rp, cols, _, status, _ = run_xattn(w, q, k, mode, tau=0.0, scores=False)
     assert status == abi.EA_OK
-    n_qb = -(-w.S // 128)
+    n_qb = -(-w.S // w.block)
     for b in range(w.B):
         for h in range(w.H_kv):
             for qb in range(n_qb):
@@ -151,11 +159,11 @@ def test_tau_one_is_a_valid_full_cover():
     rp, cols, sc, status, _ = run_xattn(w, q, k, mode, tau=1.0)
     assert status == abi.EA_OK
     qf, kf = _gpu.to_f64(q), _gpu.to_f64(k)
-    n_qb = -(-w.S // 128)
+    n_qb = -(-w.S // w.block)
     for h in range(w.H_kv):
         if _kinds(w, mode, 0, h) != wl.BLOCK_SPARSE:
             continue
-        A = ox.group_importance(qf, kf, 0, h, w.stride, 128)
+        A = ox.group_importance(qf, kf, 0, h, w.stride, w.block)
         for qb in range(n_qb):
             r = h * n_qb + qb
             check_row(cols[rp[r]:rp[r + 1]], A[qb], qb, 1.0)
@@ -179,11 +187,11 @@ def test_bad_head_mode_is_reported():
     assert status == abi.EA_ERR_BAD_LAYOUT
 
 
-@pytest.mark.parametrize("name", SMALL)
-def test_attention_over_the_selected_layout(name):
+@pytest.mark.parametrize("name,block", [(n, 128) for n in SMALL] + [(SMALL[0], 64), (SMALL[2], 64)])
+def test_attention_over_the_selected_layout(name, block):
     """The device layout goes straight into the attention call (no host round trip); the
     output matches the attention oracle on that layout."""
-    w = wl.WORKLOADS[name]
+    w = _w(name, block)
     q, k, v, _, _ = _gpu.cached_inputs(name)
     mode = _mode(w)
     rp, cols, _, status, dpat = run_xattn(w, q, k, mode, scores=False)
@@ -210,7 +218,7 @@ def test_full_size_sampled(name):
     mode = _mode(w)
     rp, cols, sc, status, dpat = run_xattn(w, q, k, mode)
     assert status == abi.EA_OK
-    n_qb = -(-w.S // 128)
+    n_qb = -(-w.S // w.block)
     assert rp[0] == 0 and np.all(np.diff(rp) >= 0)
     rng = np.random.default_rng(3)
     qbs = np.unique(np.concatenate([[0, 1, n_qb // 2, n_qb - 1], rng.integers(0, n_qb, 4)]))
@@ -219,12 +227,12 @@ def test_full_size_sampled(name):
             if _kinds(w, mode, b, h) != wl.BLOCK_SPARSE:
                 continue
             for qb in qbs:
-                lo, hi = qb * 128, min((qb + 1) * 128, w.S)
+                lo, hi = qb * w.block, min((qb + 1) * w.block, w.S)
                 kb_hi = hi
                 qs = _gpu.to_f64(q[b:b + 1, :hi])
                 ks = _gpu.to_f64(k[b:b + 1, :kb_hi])
-                a = ox.row_importance(qs, ks, 0, h, qb, w.stride, 128)
-                np.testing.assert_allclose(sc[b, h, qb, :qb + 1], a, rtol=1e-3, atol=2e-5 * 128 / w.stride)
+                a = ox.row_importance(qs, ks, 0, h, qb, w.stride, w.block)
+                np.testing.assert_allclose(sc[b, h, qb, :qb + 1], a, rtol=1e-3, atol=2e-5 * w.block / w.stride)
                 r = (b * w.H_kv + h) * n_qb + qb
                 check_row(cols[rp[r]:rp[r + 1]], a, qb, w.tau)
     # attention over the device layout, sampled rows

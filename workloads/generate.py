@@ -127,6 +127,9 @@ WORKLOADS = {w.name: w for w in [
     _w("qwen-g7-s64k-xattn", 1, 65536, 3584, 28, 4, 128, "bf16", 128, 2048, (BLOCK_SPARSE,) * 4,
        ("fixed", 2), note="FA-XA: dense heads full, sparse heads XAttention (stride 8, tau 0.9)", pos_amp=1.8,
        **_XA),
+    _w("qwen-g7-s64k-xattn-b64", 1, 65536, 3584, 28, 4, 128, "bf16", 128, 2048, (BLOCK_SPARSE,) * 4,
+       ("fixed", 2), block=64, pos_amp=1.8,
+       note="FA-XA with XAttention selecting 64-key blocks (the pages' block edge)", **_XA),
     _w("llama3-8b-s32k-xassa", 1, 32768, 4096, 32, 8, 128, "bf16", 128, 2048, (STREAMING,) * 8,
        ("fixed", 4), kinds_dense=(BLOCK_SPARSE,) * 8,
        note="XA-SSA: dense heads XAttention (stride 8, tau 0.9), sparse heads streaming", pos_amp=1.7, **_XA),
