@@ -296,7 +296,8 @@ EA_API ea_status ea_static_head_assignment(const float* scores, int L, int B, in
                                            double omega_msr, int32_t* head_mode, void* stream);
 
 /* Test hook for the failure path (no counterpart in the paper): the next
- * `launches` tensor-core attention launches make the MMA thread of their first
+ * `launches` tensor-core attention launches of layouts other than block 64
+ * (block-64 launches neither use nor consume it) make the MMA thread of their first
  * CTA wait on a barrier that nothing arrives on.  That bounded wait runs out
  * (about 2 s), the CTA drains its own copies and MMAs, frees TMEM and exits, and
  * the workspace status word reads EA_ERR_TIMEOUT; the output of that CTA's work
