@@ -171,3 +171,28 @@ def test_assignment_and_stack_argument_checks(lib):
                                  ctypes.c_void_p(0x100000), 1 << 30, None) == abi.EA_ERR_INVALID_ARG
     assert abi.ea_retrieval_workspace_size(1, 32768, 32, 8) % 256 == 0
     assert abi.ea_retrieval_workspace_size(1, 32768, 30, 8) == 0
+
+
+def _declared_arity():
+    """name -> number of parameters, parsed from include/ea.h."""
+    import re
+    text = open(abi.HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for m in re.finditer(r"EA_API\s+[\w\s\*]+?\b(ea_\w+)\s*\(([^)]*)\)", text):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_header(lib):
+    """Every ctypes signature the binding sets has the parameter count the header declares."""
+    arity = _declared_arity()
+    assert len(arity) == len(abi.declared_symbols())
+    checked = 0
+    for name, n in arity.items():
+        fn = getattr(lib, name)
+        if fn.argtypes is not None:
+            assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+            checked += 1
+    assert checked == len(arity)
