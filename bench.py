@@ -728,6 +728,7 @@ def router_bandwidth(w, hidden, weights, dev, st):
     with torch.cuda.graph(g_b):
         abi.ea_router(hidden, weights, hm, ws_b, w.n_boundary)
     for it in range(8):
+        flush.zero_()                  # as for the full-sequence replays
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(st)
         g_b.replay()
@@ -737,7 +738,17 @@ def router_bandwidth(w, hidden, weights, dev, st):
             boundary.append(a.elapsed_time(b))
     del g_b
     del flush
+    # Pooling alone: both graphs run the same projection and MLP, so the difference in time is the
+    # pooling of the rows the boundary mode skips.
+    extra_rows = max(0, w.S - 2 * w.n_boundary)
+    pool_bytes = w.B * extra_rows * w.D * hidden.element_size()
+    dt = ms - statistics.median(boundary) if boundary else 0.0
+    pool_only = {"achieved": round(pool_bytes / (dt * 1e-3) / 1e9, 1) if dt > 0 else None,
+                 "frac": round(pool_bytes / (dt * 1e-3) / 1e9 / pk["hbm"], 4) if dt > 0 else None,
+                 "bytes": int(pool_bytes), "ms": round(dt, 4),
+                 "how": "full-sequence minus boundary-mode router time (same projection and MLP in both)"}
     return {"bound": "hbm", "mode": "full-sequence pooling (n_boundary=0), whole router call as a CUDA graph",
+            "pooling_only": pool_only,
             "achieved": round(gbs, 1),
             "peak": pk["hbm"], "unit": "GB/s", "frac": round(gbs / pk["hbm"], 4), "bytes": int(bytes_),
             "ms": round(ms, 4), "boundary_mode_us": round(1e3 * statistics.median(boundary), 2)}
