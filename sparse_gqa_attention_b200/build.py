@@ -51,7 +51,10 @@ def build(force: bool = False, verbose: bool = False) -> str:
     """Compile every CUDA source of the library into libea.so (skipped when up to date)."""
     if not force and not _stale():
         return LIB
-    cmd = [nvcc(), *NVCC_FLAGS, "-shared", "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp", *sources()]
+    # A private temporary per process, then an atomic rename: ranks that build at once (one
+    # process per GPU) never write the same file, and a reader never sees a partial library.
+    tmp = f"{LIB}.tmp{os.getpid()}"
+    cmd = [nvcc(), *NVCC_FLAGS, "-shared", "-I", os.path.join(ROOT, "include"), "-o", tmp, *sources()]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd))
@@ -60,8 +63,10 @@ def build(force: bool = False, verbose: bool = False) -> str:
         sys.stdout.write(res.stdout)
         sys.stderr.write(res.stderr)
     if res.returncode != 0:
+        if os.path.exists(tmp):
+            os.remove(tmp)
         raise RuntimeError(f"nvcc failed ({res.returncode})")
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(tmp, LIB)
     return LIB
 
 
