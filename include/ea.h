@@ -143,7 +143,7 @@ EA_API ea_status ea_router_static_scratch(const void* hidden, ea_dtype dtype, in
 typedef struct {
   int n_sink;                   /* streaming sink tokens (>= 0); pages: 128        */
   int window;                   /* streaming local window incl. the query (>= 1)   */
-  int block;                    /* block edge of BLOCK_SPARSE / STREAMING_BLOCKS; 128 */
+  int block;                    /* block edge of BLOCK_SPARSE / STREAMING_BLOCKS: 64 (the pages') or 128 */
   const int32_t* bs_row_ptr;    /* device CSR [B*H_kv*ceil(S/block) + 1]; rows r = */
   const int32_t* bs_col;        /*   (b*H_kv + h)*n_qb + qb; cols sorted, with qb  */
   long long bs_nnz;             /* entries in bs_col (bounds every column read)    */
