@@ -196,3 +196,24 @@ def test_binding_signatures_match_the_header(lib):
             assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
             checked += 1
     assert checked == len(arity)
+
+
+def test_no_fallback_without_the_library(monkeypatch, tmp_path):
+    """The binding never computes on the host: without libea.so every call raises."""
+    monkeypatch.setattr(abi, "_LIB", None)
+    monkeypatch.setattr(abi, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        abi.ea_attn_workspace_size(1, 128, 8, 2)
+    with pytest.raises(RuntimeError, match="not built"):
+        abi.ea_router_workspace_size(1, 128, 256, 2, 128, 100)
+
+
+def test_host_tensors_are_refused(lib):
+    """Device pointers only: a CPU tensor is rejected before any call into the library."""
+    import torch
+    q = torch.zeros(1, 128, 8, 128, dtype=torch.bfloat16)
+    k = torch.zeros(1, 128, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(TypeError, match="CUDA tensor"):
+        abi._dev(q, "q")
+    with pytest.raises(TypeError):
+        abi.ea_retrieval_scores(q, k, 0, 1, torch.zeros(1, 8), torch.zeros(1024, dtype=torch.uint8))
