@@ -194,6 +194,7 @@ class Pattern:
 # ---------------------------------------------------------------------------
 
 def ea_router_workspace_size(B: int, S: int, D: int, H_kv: int, d: int, n_boundary: int = 100) -> int:
+    """Bytes of scratch ea_router needs (pooling and projection partial sums, MLP vectors)."""
     return int(_lib().ea_router_workspace_size(B, S, D, H_kv, d, n_boundary))
 
 
@@ -237,6 +238,7 @@ def ea_router_static_scratch(hidden: torch.Tensor, weights: dict, head_mode: tor
 # ---------------------------------------------------------------------------
 
 def ea_attn_workspace_size(B: int, S: int, H_q: int, H_kv: int) -> int:
+    """Bytes of workspace the attention calls and the sparsity reports need."""
     return int(_lib().ea_attn_workspace_size(B, S, H_q, H_kv))
 
 
@@ -269,6 +271,7 @@ def ea_hybrid_attn_prefill_chunk(q, k, v, head_mode, pattern: Pattern, o, worksp
 
 
 def ea_build_schedule(head_mode, pattern: Pattern, B, S, H_q, H_kv, d, workspace, stream=None):
+    """Device work list of live (query tile, head pair) items, longest first, into the workspace."""
     p = pattern.c_struct()
     _check(_lib().ea_build_schedule(_dev(head_mode, "head_mode", torch.int32), ctypes.byref(p), B, S, H_q, H_kv,
                                     d, _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
@@ -276,6 +279,7 @@ def ea_build_schedule(head_mode, pattern: Pattern, B, S, H_q, H_kv, d, workspace
 
 
 def ea_attn_scheduled(q, k, v, head_mode, pattern: Pattern, o, workspace, stream=None):
+    """The attention launch over the work list ea_build_schedule wrote (same head_mode and pattern)."""
     args, keep = _attn_args(q, k, v, head_mode, pattern, o, workspace, stream)
     _check(_lib().ea_attn_scheduled(*args), "ea_attn_scheduled")
 
@@ -287,6 +291,7 @@ def xattn_cols_capacity(B: int, S: int, H_kv: int, block: int = 128) -> int:
 
 
 def ea_xattn_workspace_size(B: int, S: int, H_q: int, H_kv: int, stride: int = 8, block: int = 128) -> int:
+    """Bytes of workspace ea_xattn_block_select needs at this stride and block edge."""
     return int(_lib().ea_xattn_workspace_size(B, S, H_q, H_kv, stride, block))
 
 
@@ -333,6 +338,7 @@ def ea_model_sparsity(head_mode, pattern: Pattern, L, B, S, H_q, H_kv, d, worksp
 
 
 def ea_retrieval_workspace_size(B: int, S: int, H_q: int, H_kv: int) -> int:
+    """Bytes of workspace ea_retrieval_scores needs (per-slice partial sums)."""
     return int(_lib().ea_retrieval_workspace_size(B, S, H_q, H_kv))
 
 
@@ -367,4 +373,5 @@ def ea_debug_inject_stall(launches: int):
 
 
 def ea_status_string(status: int) -> str:
+    """Static text for an ea_status code."""
     return _lib().ea_status_string(status).decode()
