@@ -11,8 +11,10 @@
 // The array is a file-scope __device__ variable: every GPU that loads the library holds
 // kStaticScratchBytes of it until the process exits.  Host code cannot use the array's
 // name as a device address, so the first call on each device looks the address up with
-// cudaGetSymbolAddress (that device current) and caches it; that first call should come
-// before any stream capture.  All calls share the one array, so calls whose kernels
+// cudaGetSymbolAddress (that device current) and caches it together with the context it
+// was found in; a later call in another context (after a device reset, or from a caller's
+// own context) looks it up again.  That first call in a context should come before any
+// stream capture.  All calls share the one array, so calls whose kernels
 // overlap on the GPU (different streams, or different host threads) race on it; order
 // them on one stream.  Nothing in it needs to start at zero: every byte a call reads was
 // written earlier in the same call.
@@ -30,22 +32,67 @@ constexpr int kMaxDevices = 64;
 __device__ __align__(256) unsigned char g_router_scratch[kStaticScratchBytes];
 
 std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
+// One cached address per device, valid for the context it was looked up in (by the
+// context's unique id, which the driver never reuses within a process): a different
+// current context (after a device reset, or a caller's own non-primary context) gets
+// the address looked up again.
+struct CachedAddress {
+  unsigned long long ctx_id;
+  void* ptr;
+};
+CachedAddress g_scratch[kMaxDevices] = {};
 
-// Device address of g_router_scratch on the current device (looked up once per device).
+typedef int (*CtxGetCurrentFn)(void**);                    // the driver's cuCtxGetCurrent
+typedef int (*CtxGetIdFn)(void*, unsigned long long*);     // the driver's cuCtxGetId
+
+template <typename F>
+F driver_fn(const char* name) {
+  void* f = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion(name, &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<F>(f);
+  return nullptr;
+}
+
+// Unique id of the calling thread's current context; false when there is none yet.
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_ctx = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    get_ctx = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  });
+  void* ctx = nullptr;
+  if (!get_ctx || !get_id || get_ctx(&ctx) != 0 || ctx == nullptr) return false;
+  return get_id(ctx, id) == 0;
+}
+
+// Device address of g_router_scratch in the current device's current context.
 ea_status scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return EA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return EA_ERR_UNSUPPORTED;
+  unsigned long long id = 0;
+  const bool have_ctx = current_context_id(&id);
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_router_scratch) != cudaSuccess || p == nullptr) return EA_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
+  if (have_ctx && g_scratch[dev].ptr != nullptr && g_scratch[dev].ctx_id == id) {
+    *out = g_scratch[dev].ptr;
+    return EA_OK;
   }
-  *out = g_scratch_ptr[dev];
+  // First call in this context (the lookup also starts the runtime's context on a thread
+  // that has none yet, so the context is read again afterwards).
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_router_scratch) != cudaSuccess || p == nullptr) return EA_ERR_CUDA;
+  if (!current_context_id(&id)) return EA_ERR_CUDA;
+  g_scratch[dev].ctx_id = id;
+  g_scratch[dev].ptr = p;
+  *out = p;
   return EA_OK;
 }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
 
@@ -62,6 +109,8 @@ extern "C" ea_status ea_router_static_scratch(const void* hidden, ea_dtype dtype
   if (D % (dtype == EA_DT_BF16 ? 8 : 4) != 0 || (reinterpret_cast<uintptr_t>(hidden) & 15u) != 0)
     return EA_ERR_INVALID_ARG;
   if ((size_t)D * sizeof(float) + 12u * d * sizeof(float) > 200u * 1024u) return EA_ERR_UNSUPPORTED;
+  if (!aligned16(w->w_k) || !aligned16(w->w_t1) || !aligned16(w->w_t2) || !aligned16(w->w_r1) || !aligned16(w->w_o))
+    return EA_ERR_INVALID_ARG;
   // The problem's scratch must fit the fixed array.
   if (ea::router_workspace_bytes(B, S, D, H_kv, d, prm->n_boundary) > kStaticScratchBytes) return EA_ERR_INVALID_ARG;
   void* scratch = nullptr;

@@ -18,7 +18,7 @@ def lib():
 
 def test_every_declared_symbol_is_exported(lib):
     names = abi.declared_symbols()
-    assert len(names) == 18
+    assert len(names) == 20
     for n in names:
         assert hasattr(lib, n), n
 
@@ -217,3 +217,16 @@ def test_host_tensors_are_refused(lib):
         abi._dev(q, "q")
     with pytest.raises(TypeError):
         abi.ea_retrieval_scores(q, k, 0, 1, torch.zeros(1, 8), torch.zeros(1024, dtype=torch.uint8))
+
+
+def test_static_scratch_refusal_needs_no_gpu(lib):
+    """ea_router_static_scratch refuses a problem beyond its fixed array on the host, before
+    any CUDA call (checked in a child process that sees no GPU, so nothing can launch)."""
+    from tests._static_scratch import REFUSED, refusal_without_a_gpu
+    import re
+    text = open(abi.HEADER_PATH).read()
+    m = re.search(r"#define EA_ROUTER_STATIC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", text)
+    assert m and int(m.group(1)) << int(m.group(2)) == abi.ROUTER_STATIC_SCRATCH_BYTES
+    r = REFUSED
+    assert abi.ea_router_workspace_size(r["B"], r["S"], r["D"], r["H_kv"], r["d"], 100) > abi.ROUTER_STATIC_SCRATCH_BYTES
+    assert refusal_without_a_gpu() == abi.EA_ERR_INVALID_ARG

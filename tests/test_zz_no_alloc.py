@@ -8,8 +8,6 @@ on two calls in a row (the second call reuses the array the first one left
 behind), and a problem whose scratch exceeds the array must be refused before
 any launch.  This file is collected last so a failure here never hides another.
 """
-import ctypes
-
 import numpy as np
 import pytest
 import torch
@@ -17,6 +15,7 @@ import torch
 import workloads as wl
 from sparse_gqa_attention_b200 import abi
 from tests import _gpu
+from tests._static_scratch import REFUSED, refusal_without_a_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -48,12 +47,22 @@ def test_matches_workspace_router_twice(name, n_boundary):
 
 
 def test_refuses_problems_beyond_the_scratch_array():
-    lib = abi._lib()
-    fake = ctypes.c_void_p(0x10000)   # never dereferenced: the size check fails on the host first
-    w = abi.RouterWeights(*([fake] * 9))
-    prm = abi.RouterParams(100)
-    # 64 samples x D = 32768: the pooled states alone need 8 MiB plus partial sums.
-    assert abi.ea_router_workspace_size(64, 1000, 32768, 8, 128, 100) > (8 << 20)
-    st = lib.ea_router_static_scratch(fake, abi.EA_DT_BF16, 64, 1000, 32768, 8, 128, ctypes.byref(w),
-                                      ctypes.byref(prm), fake, None, None)
-    assert st == abi.EA_ERR_INVALID_ARG
+    r = REFUSED
+    assert abi.ea_router_workspace_size(r["B"], r["S"], r["D"], r["H_kv"], r["d"], 100) > abi.ROUTER_STATIC_SCRATCH_BYTES
+    # First on a process without a GPU, where nothing can be launched ...
+    assert refusal_without_a_gpu() == abi.EA_ERR_INVALID_ARG
+    # ... then here, with real device buffers of the refused problem's sizes (hidden 4 MB,
+    # W_k 64 MB), so that every input pointer is valid memory.
+    B, S, D, H_kv, d = r["B"], r["S"], r["D"], r["H_kv"], r["d"]
+    hidden = torch.zeros(B, S, D, dtype=torch.bfloat16, device="cuda")
+    weights = {"w_k": torch.zeros(D, H_kv * d, dtype=torch.bfloat16, device="cuda"),
+               "w_t1": torch.zeros(4 * d, d, device="cuda"), "b_t1": torch.zeros(4 * d, device="cuda"),
+               "w_t2": torch.zeros(d, 4 * d, device="cuda"), "b_t2": torch.zeros(d, device="cuda"),
+               "w_r1": torch.zeros(4 * d, 2 * d, device="cuda"), "b_r1": torch.zeros(4 * d, device="cuda"),
+               "w_o": torch.zeros(H_kv, 4 * d, device="cuda"), "b_o": torch.zeros(H_kv, device="cuda")}
+    hm = torch.full((B, H_kv), -1, dtype=torch.int32, device="cuda")
+    with pytest.raises(abi.EAError) as e:
+        abi.ea_router_static_scratch(hidden, weights, hm, 100)
+    assert e.value.status == abi.EA_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert (hm == -1).all()            # nothing was written
