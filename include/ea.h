@@ -106,13 +106,23 @@ EA_API size_t ea_router_workspace_size(int B, int S, int D, int H_kv, int d, int
 
 /* Router for one layer.  hidden: device [B, S, D] in `dtype`
  * (D % 8 == 0 for bf16, D % 4 == 0 for f32); d in {64, 128};
- * 1 <= H_kv <= EA_MAX_KV_HEADS.  Writes head_mode [B, H_kv] (device int32,
- * 0 dense / 1 sparse) and, when `logits` is not NULL, z [B, H_kv] (device
- * float).  Arithmetic is fp32. */
+ * 1 <= H_kv <= EA_MAX_KV_HEADS; w_k, w_t1, w_t2, w_r1 and w_o 16-byte
+ * aligned.  Writes head_mode [B, H_kv] (device int32, 0 dense / 1 sparse)
+ * and, when `logits` is not NULL, z [B, H_kv] (device float).  Arithmetic is
+ * fp32 in fixed summation orders (repeated calls give identical results).
+ * The workspace needs no zero fill. */
 EA_API ea_status ea_router(const void* hidden, ea_dtype dtype, int B, int S, int D, int H_kv, int d,
                     const ea_router_weights* weights, const ea_router_params* params,
                     int32_t* head_mode, float* logits,
                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* Router pooling alone (the first step above): hbar [B, D] (device float) =
+ * mean of hidden[b, t, :] over the pooled tokens, with the same pooling rule,
+ * alignment and dtype contract as ea_router.  Scratch: a workspace of
+ * ea_router_pool_workspace_size bytes (256-byte aligned, no zero fill). */
+EA_API size_t ea_router_pool_workspace_size(int B, int S, int D, int n_boundary);
+EA_API ea_status ea_router_pool(const void* hidden, ea_dtype dtype, int B, int S, int D, int n_boundary,
+                                float* hbar, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Router with library-owned scratch.  The paper has no counterpart: this is an
  * interface for callers that cannot allocate device memory — a runtime or plugin
@@ -123,8 +133,9 @@ EA_API ea_status ea_router(const void* hidden, ea_dtype dtype, int B, int S, int
  * inside the library, held on every GPU that loads it until the process exits.
  * It allocates nothing (no cudaMalloc, cudaFree or allocating library call).
  * Problems whose scratch (ea_router_workspace_size) exceeds the array return
- * EA_ERR_INVALID_ARG before any launch.  The first call on each device looks
- * up the array's device address; make that first call before any stream
+ * EA_ERR_INVALID_ARG before any launch.  The first call in each context (per
+ * device; again after a device reset or in a caller's own context) looks up
+ * the array's device address; make that first call before any stream
  * capture.  All calls share the array: calls that overlap on the GPU race, so
  * order them on one stream.  Nothing in the array needs to start at zero. */
 #define EA_ROUTER_STATIC_SCRATCH_BYTES ((size_t)8 << 20)

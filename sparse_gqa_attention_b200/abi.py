@@ -24,6 +24,7 @@ EA_OK, EA_ERR_INVALID_ARG, EA_ERR_UNSUPPORTED, EA_ERR_CUDA, EA_ERR_TIMEOUT, EA_E
 EA_DT_F32, EA_DT_BF16 = 0, 1
 EA_FULL, EA_STREAMING, EA_BLOCK_SPARSE = 0, 1, 2
 MAX_KV_HEADS = 64
+ROUTER_STATIC_SCRATCH_BYTES = 8 << 20   # EA_ROUTER_STATIC_SCRATCH_BYTES
 
 
 class EAError(RuntimeError):
@@ -69,6 +70,11 @@ def _lib():
         lib.ea_router_workspace_size.argtypes = [c_int, c_int, c_int, c_int, c_int, c_int]
         lib.ea_attn_workspace_size.restype = c_size_t
         lib.ea_attn_workspace_size.argtypes = [c_int, c_int, c_int, c_int]
+        lib.ea_router_pool_workspace_size.restype = c_size_t
+        lib.ea_router_pool_workspace_size.argtypes = [c_int, c_int, c_int, c_int]
+        lib.ea_router_pool.restype = st
+        lib.ea_router_pool.argtypes = [c_void_p, c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_size_t,
+                                       c_void_p]
         lib.ea_router.restype = st
         lib.ea_router.argtypes = [c_void_p, c_int, c_int, c_int, c_int, c_int, c_int,
                                   POINTER(RouterWeights), POINTER(RouterParams), c_void_p, c_void_p,
@@ -213,6 +219,21 @@ def ea_router(hidden: torch.Tensor, weights: dict, head_mode: torch.Tensor, work
                               _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
                               _stream(stream))
     _check(status, "ea_router")
+
+
+def ea_router_pool_workspace_size(B: int, S: int, D: int, n_boundary: int = 100) -> int:
+    """Bytes of scratch ea_router_pool needs (pooling partial sums)."""
+    return int(_lib().ea_router_pool_workspace_size(B, S, D, n_boundary))
+
+
+def ea_router_pool(hidden: torch.Tensor, hbar: torch.Tensor, workspace: torch.Tensor, n_boundary: int = 100,
+                   stream=None):
+    """hbar[B, D] (float32, device) <- mean of hidden[B, S, D] over the pooled tokens."""
+    B, S, D = hidden.shape
+    status = _lib().ea_router_pool(_dev(hidden, "hidden"), _dtype_code(hidden), B, S, D, n_boundary,
+                                   _dev(hbar, "hbar", torch.float32), _dev(workspace, "workspace"),
+                                   workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(status, "ea_router_pool")
 
 
 def ea_router_static_scratch(hidden: torch.Tensor, weights: dict, head_mode: torch.Tensor, n_boundary: int = 100,

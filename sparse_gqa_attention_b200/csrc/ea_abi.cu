@@ -70,6 +70,11 @@ ea_status check_attn_data(const void* q, const void* k, const void* v, const voi
   return EA_ERR_INVALID_ARG;
 }
 
+// The router reads its weight matrices with 16-byte loads.
+bool router_weights_aligned(const ea_router_weights* w) {
+  return aligned16(w->w_k) && aligned16(w->w_t1) && aligned16(w->w_t2) && aligned16(w->w_r1) && aligned16(w->w_o);
+}
+
 ea_status check_ws(const void* ws, size_t bytes, size_t need) {
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return EA_ERR_INVALID_ARG;
   return bytes >= need ? EA_OK : EA_ERR_INVALID_ARG;
@@ -84,6 +89,11 @@ size_t ea_router_workspace_size(int B, int S, int D, int H_kv, int d, int n_boun
   return router_workspace_bytes(B, S, D, H_kv, d, n_boundary);
 }
 
+size_t ea_router_pool_workspace_size(int B, int S, int D, int n_boundary) {
+  if (B < 1 || S < 1 || D < 1) return 0;
+  return router_pool_workspace_bytes(B, S, D, n_boundary);
+}
+
 ea_status ea_router(const void* hidden, ea_dtype dtype, int B, int S, int D, int H_kv, int d,
                     const ea_router_weights* w, const ea_router_params* prm, int32_t* head_mode, float* logits,
                     void* workspace, size_t workspace_bytes, void* stream) {
@@ -96,9 +106,21 @@ ea_status ea_router(const void* hidden, ea_dtype dtype, int B, int S, int D, int
   if (dtype != EA_DT_BF16 && dtype != EA_DT_F32) return EA_ERR_INVALID_ARG;
   if (D % (dtype == EA_DT_BF16 ? 8 : 4) != 0 || !aligned16(hidden)) return EA_ERR_INVALID_ARG;
   if ((size_t)D * sizeof(float) + 12u * d * sizeof(float) > 200u * 1024u) return EA_ERR_UNSUPPORTED;
+  if (!router_weights_aligned(w)) return EA_ERR_INVALID_ARG;
   if (ea_status s = check_ws(workspace, workspace_bytes, router_workspace_bytes(B, S, D, H_kv, d, prm->n_boundary)))
     return s;
   return launch_router(hidden, dtype, B, S, D, H_kv, d, w, prm, head_mode, logits, workspace, as_stream(stream));
+}
+
+ea_status ea_router_pool(const void* hidden, ea_dtype dtype, int B, int S, int D, int n_boundary, float* hbar,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (!hidden || !hbar) return EA_ERR_INVALID_ARG;
+  if (B < 1 || S < 1 || D < 1) return EA_ERR_INVALID_ARG;
+  if (dtype != EA_DT_BF16 && dtype != EA_DT_F32) return EA_ERR_INVALID_ARG;
+  if (D % (dtype == EA_DT_BF16 ? 8 : 4) != 0 || !aligned16(hidden)) return EA_ERR_INVALID_ARG;
+  if ((long long)B * D > (1LL << 31) - 256) return EA_ERR_UNSUPPORTED;
+  if (ea_status s = check_ws(workspace, workspace_bytes, router_pool_workspace_bytes(B, S, D, n_boundary))) return s;
+  return launch_router_pool(hidden, dtype, B, S, D, n_boundary, hbar, workspace, as_stream(stream));
 }
 
 size_t ea_attn_workspace_size(int B, int S, int H_q, int H_kv) {

@@ -12,6 +12,9 @@ size_t router_workspace_bytes(int B, int S, int D, int H_kv, int d, int n_bounda
 ea_status launch_router(const void* hidden, ea_dtype dtype, int B, int S, int D, int H_kv, int d,
                         const ea_router_weights* w, const ea_router_params* prm, int32_t* head_mode,
                         float* logits, void* workspace, cudaStream_t st);
+size_t router_pool_workspace_bytes(int B, int S, int D, int n_boundary);
+ea_status launch_router_pool(const void* hidden, ea_dtype dtype, int B, int S, int D, int n_boundary, float* hbar,
+                             void* workspace, cudaStream_t st);
 
 size_t attn_workspace_bytes(int B, int S, int H_q, int H_kv);
 int n_pairs(int H_q, int H_kv);

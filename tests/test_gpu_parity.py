@@ -58,6 +58,42 @@ def test_router_full_sequence_pooling(name):
     np.testing.assert_array_equal(hm[sure], m_ref[sure])
 
 
+@pytest.mark.parametrize("name,n_boundary", [(n, nb) for n in SMALL[:4] + ["llama3-8b-b4-s16k-mixed"] for nb in (100, 0)]
+                         + [("llama3-8b-s32k-streaming", 100), ("llama3-8b-s32k-streaming", 0)])
+def test_router_pooling_matches_oracle(name, n_boundary):
+    """ea_router_pool (the pooling step alone) against the oracle's pooled mean."""
+    w = wl.WORKLOADS[name]
+    hidden = wl.hidden_states(w)
+    hb = torch.full((w.B, w.D), float("nan"), dtype=torch.float32, device="cuda")
+    ws = torch.empty(abi.ea_router_pool_workspace_size(w.B, w.S, w.D, n_boundary), dtype=torch.uint8, device="cuda")
+    abi.ea_router_pool(_gpu.to_dev(hidden, w.dtype), hb, ws, n_boundary)
+    torch.cuda.synchronize()
+    ref = oracle.router.pool_hidden(_gpu.to_f64(hidden), n_boundary)
+    np.testing.assert_allclose(hb.cpu().numpy(), ref, rtol=1e-4, atol=1e-5)
+
+
+@pytest.mark.parametrize("name", ["small-mixed-g4-s1000", "llama3-8b-b4-s16k-mixed"])
+def test_router_repeats_bit_for_bit(name):
+    """Fixed summation orders: the same inputs give the same logits on every call, also
+    with a workspace that was not zero-filled."""
+    w = wl.WORKLOADS[name]
+    _, _, _, hidden, weights = _gpu.cached_inputs(name)
+    hid = _gpu.to_dev(hidden, w.dtype)
+    wd = {k: _gpu.to_dev(v, w.dtype) for k, v in weights.items()}
+    zs = []
+    for fill in (0, 255):
+        ws = torch.full((abi.ea_router_workspace_size(w.B, w.S, w.D, w.H_kv, w.d, w.n_boundary),), fill,
+                        dtype=torch.uint8, device="cuda")
+        hm = torch.full((w.B, w.H_kv), -1, dtype=torch.int32, device="cuda")
+        z = torch.full((w.B, w.H_kv), float("nan"), dtype=torch.float32, device="cuda")
+        for _ in range(2):
+            abi.ea_router(hid, wd, hm, ws, w.n_boundary, logits=z)
+            zs.append(z.clone())
+    torch.cuda.synchronize()
+    for z in zs[1:]:
+        assert torch.equal(z, zs[0])
+
+
 # ---------------------------------------------------------------------------- attention
 
 @pytest.mark.parametrize("name", SMALL)
