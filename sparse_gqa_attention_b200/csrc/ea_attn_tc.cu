@@ -8,19 +8,22 @@
 // o[b, i, h_q, :]; all kinds run in this one launch, fed by the device-built
 // work list, and only the live key tiles of each head are visited.
 //
-// Design (B200): persistent CTAs, one per SM, walking the cost-sorted work list in
-// a snake order.  A work item is 128 query rows of two query heads of one KV
+// Design (B200): persistent CTAs, one per SM, claiming items of the cost-sorted work
+// list (longest first) at run time.  A work item is 128 query rows of two query heads of one KV
 // group (two "slots"), so every K/V tile brought into shared memory feeds two
 // 128x128 products.  Warp roles, 384 threads:
 //   warp 0      TMA producer: Q tiles of both slots, then the K and V tiles of the
 //               live key tiles through one 3-slot ring in the order the MMAs use
 //               them (K0, K1, V0, K2, V1, ...), 128-byte swizzle, 2 boxes of 64
 //               columns per 128x128 tile.  No cluster multicast.
-//   warp 1      TMEM owner and MMA issuer (one thread): S_s = Q_s K^T into TMEM
-//               (M=N=128, K=16 steps), O_s += P_s V with P_s and V both read from
-//               shared memory (V as an MN-major operand).  For key tile j it issues
-//               S(j+1) before O += P(j) V(j), so the tensor pipe computes the next
-//               scores while the softmax works on the current ones.
+//   warp 1      TMEM owner and Q K^T issuer (one thread): S_s = Q_s K^T into TMEM
+//               (M=N=128, K=16 steps); it runs a key tile ahead of the softmax, so
+//               the tensor pipe computes the next scores while the softmax works on
+//               the current ones.
+//   warp 2      P V issuer (one thread): O_s += P_s V with P_s and V both read from
+//               shared memory (V as an MN-major operand).  Two issuing threads on
+//               two SM sub-partitions: a single thread issuing both products, with
+//               their barrier waits, could not keep the tensor pipe fed.
 //   warps 4-7   softmax for slot 0, warps 8-11 for slot 1: one thread per query
 //               row (its TMEM lane).  Loads S from TMEM and releases it at once,
 //               applies the element rule only on boundary tiles, keeps a running
@@ -59,11 +62,15 @@ constexpr uint32_t OFF_BAR = OFF_KV + NKV * kTileBytes;
 enum : int {
   B_QFULL = 0, B_QEMPTY = 2, B_KVFULL = 4, B_KVEMPTY = B_KVFULL + NKV, B_SFULL = B_KVEMPTY + NKV,
   B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2, B_PVDONE = B_PFULL + 2, B_OFULL = B_PVDONE + 2,
-  B_FIN = B_OFULL + 2, B_NEVER = B_FIN + 1, N_BAR = B_NEVER + 1
+  B_FIN = B_OFULL + 2, B_FIN2 = B_FIN + 1, B_TOK = B_FIN2 + 1, B_IFULL = B_TOK + 8, B_IEMPTY = B_IFULL + 2,
+  B_NEVER = B_IEMPTY + 2, N_BAR = B_NEVER + 1
 };
 constexpr uint32_t OFF_TMEM = OFF_BAR + N_BAR * 8;
 constexpr uint32_t OFF_ABORT = OFF_TMEM + 4;
-constexpr uint32_t kSmemBytes = OFF_ABORT + 4 + 1024;  // + slack to align the base to 1024
+constexpr uint32_t OFF_IRING = OFF_ABORT + 4;          // 2 claimed item indices
+constexpr uint32_t kSmemBytes = OFF_IRING + 8 + 1024;  // + slack to align the base to 1024
+// Roles that read every claimed item: Q K^T issuer, P V issuer and the 8 softmax warps.
+constexpr uint32_t kItemReaders = 10;
 static_assert(kSmemBytes <= 232448, "shared memory beyond the 227 KB a CTA may use");
 constexpr uint32_t kTmemCols = 512;
 __device__ __forceinline__ uint32_t col_s(int s) { return 128u * s; }        // S_s (and P_s) columns
@@ -118,9 +125,24 @@ struct Item {
   bool two;
 };
 
-__device__ __forceinline__ int item_index(int it, int cta, int ncta) {
-  return it * ncta + ((it & 1) ? (ncta - 1 - cta) : cta);
-}
+// Work items are claimed at run time: the producer takes the next index of the cost-sorted
+// list (longest first) from a counter in the workspace whenever its CTA can start another
+// item, and passes it to the other roles through a 2-entry ring in shared memory; -1 ends
+// the list.  Greedy longest-first claiming keeps the CTAs' finishing times close.
+struct ItemRing {
+  volatile int* slot;   // 2 entries
+  int k;                // items read so far
+  // Next item index for a reader role (-1: done or aborted).  `arrive` is true for the one
+  // thread of the role that signals the entry as read.
+  __device__ int next(const Ctx& c, bool arrive) {
+    const int e = k & 1;
+    const bool ok = wait(c, c.bar(B_IFULL + e), (k >> 1) & 1);
+    const int idx = ok ? slot[e] : -1;
+    if (ok && arrive) mbar_arrive(c.bar(B_IEMPTY + e));
+    ++k;
+    return idx;
+  }
+};
 
 __device__ __forceinline__ Item load_item(const int4* items, int idx, const PatternDev& p,
                                           const int32_t* head_mode, int H_kv, int G) {
@@ -157,9 +179,10 @@ __device__ __forceinline__ uint64_t v_desc(uint32_t tile, int kk) {
   return sdesc_sw128(tile + (uint32_t)kk * 2048u, kBoxBytes, 1024u);
 }
 
-// S_s = Q_s K^T for the key tile at kt, once the softmax has loaded the previous S_s.
+// S_s = Q_s K^T for the key tile at kt, once the softmax has loaded the previous S_s.  After
+// the item's last key tile (last), Q_s is released once the product has read it.
 __device__ __forceinline__ bool issue_qk(const Ctx& c, uint32_t tmem, uint32_t base, int s, uint32_t kt,
-                                         int& s_cnt) {
+                                         int& s_cnt, bool last) {
   if (s_cnt > 0 && !wait(c, c.bar(B_SFREE + s), (s_cnt - 1) & 1)) return false;
   fence_after_sync();
   const uint32_t qt = base + OFF_Q + s * kTileBytes;
@@ -167,6 +190,7 @@ __device__ __forceinline__ bool issue_qk(const Ctx& c, uint32_t tmem, uint32_t b
   for (int kk = 0; kk < HD / 16; ++kk)
     mma_ss(tmem + col_s(s), qk_desc(qt, kk), qk_desc(kt, kk), IDESC_QK, kk > 0 ? 1u : 0u);
   commit(c.bar(B_SFULL + s));
+  if (last) commit(c.bar(B_QEMPTY + s));
   ++s_cnt;
   return true;
 }
@@ -182,10 +206,7 @@ __device__ __forceinline__ bool issue_pv(const Ctx& c, uint32_t tmem, uint32_t b
   for (int kk = 0; kk < BN / 16; ++kk)
     mma_ss(tmem + col_o(s), qk_desc(pt, kk), v_desc(vt, kk), IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
   commit(c.bar(B_PVDONE + s));
-  if (last) {
-    commit(c.bar(B_OFULL + s));
-    commit(c.bar(B_QEMPTY + s));
-  }
+  if (last) commit(c.bar(B_OFULL + s));
   return true;
 }
 
@@ -223,11 +244,13 @@ __device__ __forceinline__ void ex2_pair_fma(uint64_t t2, float& r0, float& r1) 
 
 // One 128-key tile of one query row: running max (raised only past kRescaleLog2),
 // row sum, and P = exp2(scale*log2e*s - max) as bf16 pairs in pk (pk[j] holds keys
-// 2j, 2j+1).  kMode 0: every key live; 1: causal rule; 2: streaming rule.  Returns
-// the factor O must be multiplied by (1 when the max was not raised).
-template <int kMode>
+// 2j, 2j+1).  kMode 0: every key live; 1: causal rule; 2: streaming rule.  The
+// exponentials run inside this warp's MUFU turn (tok).  Returns the factor O must be
+// multiplied by (1 when the max was not raised).
+template <int kMode, typename Tok>
 __device__ __forceinline__ float softmax_tile(const float (&x)[BN], int lim, int sink_lim, int win_lim,
-                                              float scale_log2, float& m_ref, float& l, uint32_t (&pk)[BN / 2]) {
+                                              float scale_log2, float& m_ref, float& l, uint32_t (&pk)[BN / 2],
+                                              Tok& tok) {
   auto live = [&](int e) {
     if (kMode == 0) return true;
     if (kMode == 1) return e <= lim;
@@ -251,7 +274,9 @@ __device__ __forceinline__ float softmax_tile(const float (&x)[BN], int lim, int
     l *= f;
     m_ref = mts;
   }
-  const float sub = (m_ref == -INFINITY) ? 0.f : m_ref;
+  // The exponentials start once this warp holds its sub-partition's MUFU turn; `sub` takes
+  // a zero that only exists after the wait, so no exponential is scheduled before it.
+  const float sub = ((m_ref == -INFINITY) ? 0.f : m_ref) + tok.acquire();
   const uint64_t scale2 = f2_pack(scale_log2, scale_log2), nsub2 = f2_pack(-sub, -sub);
   uint64_t l2 = f2_pack(0.f, 0.f);
 #pragma unroll
@@ -275,6 +300,7 @@ __device__ __forceinline__ float softmax_tile(const float (&x)[BN], int lim, int
   float la, lb;
   f2_unpack(l2, la, lb);
   l += la + lb;
+  tok.release(l);   // after the last exponential (the row sum depends on all of them)
   return f;
 }
 
@@ -293,6 +319,31 @@ __device__ __forceinline__ void store_p_row(uint32_t p_tile, int row, const uint
     }
   }
 }
+
+// MUFU turns of the two softmax warps that share an SM sub-partition (slot 0 and slot 1 of
+// TMEM lane quadrant q): their exponential phases alternate, so each warp's loads, row max
+// and P stores overlap the other's exponentials instead of both contending for the MUFU unit
+// at once and leaving it idle together.  Slot 0 goes first; turn k of slot 0 waits for turn
+// k-1 of slot 1, turn k of slot 1 for turn k of slot 0 (bounded waits, so a warp is never
+// more than one phase ahead).  Items with a single query head take no turns.
+struct MufuTurn {
+  const Ctx* c;
+  uint32_t mine, theirs;   // barrier this warp arrives on / waits on
+  int slot, n;             // turns taken so far
+  bool on, ok;
+  __device__ float acquire() {
+    if (on && (slot == 1 || n > 0)) ok = wait(*c, theirs, (slot == 1 ? n : n - 1) & 1) && ok;
+    float z;
+    asm volatile("mov.b32 %0, 0;" : "=f"(z) :: "memory");
+    return z;
+  }
+  __device__ void release(float dep) {
+    if (!on) return;
+    asm volatile("" ::"f"(dep) : "memory");
+    mbar_arrive(mine);
+    ++n;
+  }
+};
 
 __global__ void __launch_bounds__(kThreads, 1)
 hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -317,7 +368,9 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     tma_prefetch_map(&tm_v);
     for (int i = 0; i < N_BAR; ++i) {
       const bool softmax_arrive = (i >= B_SFREE && i < B_SFREE + 2) || (i >= B_PFULL && i < B_PFULL + 2);
-      mbar_init(c.bar(i), softmax_arrive ? 128u : 1u);
+      const bool token = i >= B_TOK && i < B_TOK + 8;   // one softmax warp arrives
+      const bool item_read = i >= B_IEMPTY && i < B_IEMPTY + 2;
+      mbar_init(c.bar(i), softmax_arrive ? 128u : token ? 32u : item_read ? kItemReaders : 1u);
     }
     *c.abort_flag = 0;
     fence_mbar_init();
@@ -348,9 +401,17 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         ++kv;
         return true;
       };
+      volatile int* ring = reinterpret_cast<volatile int*>(gbase + OFF_IRING);
       for (int it = 0; ok; ++it) {
-        const int idx = item_index(it, blockIdx.x, gridDim.x);
-        if (idx >= n_items) break;
+        // Claim the next item once the readers are done with this ring entry's last use.
+        const int e = it & 1;
+        ok = wait(c, c.bar(B_IEMPTY + e), ((it >> 1) & 1) ^ 1);
+        if (!ok) break;
+        int idx = (int)atomicAdd(hdr + kWsClaim / 4, 1u);
+        if (idx >= n_items) idx = -1;
+        ring[e] = idx;
+        mbar_arrive(c.bar(B_IFULL + e));
+        if (idx < 0) break;
         const Item I = load_item(items, idx, p, head_mode, H_kv, G);
         if (I.n == 0) continue;
 #pragma unroll
@@ -383,15 +444,29 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (q_use[s] > 0) wait_drain(c, c.bar(B_QFULL + s), (q_use[s] - 1) & 1);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ Q K^T issuer
+    // Walks the ring in the producer's order; takes the K entries, skips the V entries.
     if (lane == 0) {
-      int q_use[2] = {0, 0}, s_cnt[2] = {0, 0}, p_cnt[2] = {0, 0};
+      int q_use[2] = {0, 0}, s_cnt[2] = {0, 0};
       int kv = 0;
       // Test hook for the timeout path: CTA 0 first waits on a barrier nothing arrives on.
       bool ok = !(inject_stall && blockIdx.x == 0) || wait(c, c.bar(B_NEVER), 0);
-      for (int it = 0; ok; ++it) {
-        const int idx = item_index(it, blockIdx.x, gridDim.x);
-        if (idx >= n_items) break;
+      // S of key tile jj (both slots); the ring slot is released once both products finish.
+      auto qk_tile = [&](const Item& I, int jj) -> bool {
+        const int slot = kv % NKV;
+        if (!wait(c, c.bar(B_KVFULL + slot), (kv / NKV) & 1)) return false;
+        const uint32_t kt = base + OFF_KV + slot * kTileBytes;
+        const bool last = jj + 1 == I.n;
+        if (!issue_qk(c, tmem, base, 0, kt, s_cnt[0], last)) return false;
+        if (I.two && !issue_qk(c, tmem, base, 1, kt, s_cnt[1], last)) return false;
+        commit(c.bar(B_KVEMPTY + slot));
+        ++kv;
+        return true;
+      };
+      ItemRing ir{reinterpret_cast<volatile int*>(gbase + OFF_IRING), 0};
+      while (ok) {
+        const int idx = ir.next(c, true);
+        if (idx < 0) break;
         const Item I = load_item(items, idx, p, head_mode, H_kv, G);
         if (I.n == 0) continue;
         ok = wait(c, c.bar(B_QFULL + 0), q_use[0] & 1);
@@ -400,35 +475,36 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           ok = ok && wait(c, c.bar(B_QFULL + 1), q_use[1] & 1);
           ++q_use[1];
         }
-        // S of the item's first key tile; the ring slot is released once both products finish.
-        {
-          const int slot = kv % NKV;
-          ok = ok && wait(c, c.bar(B_KVFULL + slot), (kv / NKV) & 1);
-          if (ok) {
-            const uint32_t kt = base + OFF_KV + slot * kTileBytes;
-            ok = issue_qk(c, tmem, base, 0, kt, s_cnt[0]);
-            if (ok && I.two) ok = issue_qk(c, tmem, base, 1, kt, s_cnt[1]);
-            if (ok) commit(c.bar(B_KVEMPTY + slot));
-            ++kv;
-          }
-        }
+        ok = ok && qk_tile(I, 0);
         for (int jj = 0; jj < I.n && ok; ++jj) {
-          const bool last = jj + 1 == I.n;
-          if (!last) {   // the next scores first: they run while the softmax works on tile jj
-            const int slot = kv % NKV;
-            ok = wait(c, c.bar(B_KVFULL + slot), (kv / NKV) & 1);
-            if (!ok) break;
-            const uint32_t kt = base + OFF_KV + slot * kTileBytes;
-            ok = issue_qk(c, tmem, base, 0, kt, s_cnt[0]);
-            if (ok && I.two) ok = issue_qk(c, tmem, base, 1, kt, s_cnt[1]);
-            if (!ok) break;
-            commit(c.bar(B_KVEMPTY + slot));
-            ++kv;
-          }
+          if (jj + 1 < I.n) ok = qk_tile(I, jj + 1);   // ring order: K(jj+1), then V(jj)
+          ++kv;                                       // V(jj): the P V issuer's entry
+        }
+      }
+      commit(c.bar(B_FIN));                       // every MMA issued here has completed
+      wait_drain(c, c.bar(B_FIN), 0);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ P V issuer
+    // Walks the ring in the producer's order; takes the V entries, skips the K entries.
+    if (lane == 0) {
+      int p_cnt[2] = {0, 0};
+      int kv = 0;
+      bool ok = true;
+      ItemRing ir{reinterpret_cast<volatile int*>(gbase + OFF_IRING), 0};
+      while (ok) {
+        const int idx = ir.next(c, true);
+        if (idx < 0) break;
+        const Item I = load_item(items, idx, p, head_mode, H_kv, G);
+        if (I.n == 0) continue;
+        ++kv;                                         // K(0)
+        for (int jj = 0; jj < I.n && ok; ++jj) {
+          if (jj + 1 < I.n) ++kv;                     // K(jj+1)
           const int slot = kv % NKV;
           ok = wait(c, c.bar(B_KVFULL + slot), (kv / NKV) & 1);
           if (!ok) break;
           const uint32_t vt = base + OFF_KV + slot * kTileBytes;
+          const bool last = jj + 1 == I.n;
           ok = issue_pv(c, tmem, base, 0, vt, jj > 0, last, p_cnt[0]);
           if (ok && I.two) ok = issue_pv(c, tmem, base, 1, vt, jj > 0, last, p_cnt[1]);
           if (!ok) break;
@@ -436,8 +512,8 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           ++kv;
         }
       }
-      commit(c.bar(B_FIN));                       // every MMA issued here has completed
-      wait_drain(c, c.bar(B_FIN), 0);
+      commit(c.bar(B_FIN2));
+      wait_drain(c, c.bar(B_FIN2), 0);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax slots
@@ -448,11 +524,22 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const uint32_t p_tile = base + OFF_P + s * kTileBytes;
     int s_cnt = 0, p_cnt = 0, o_cnt = 0;
     bool ok = true;
-    for (int it = 0; ok; ++it) {
-      const int idx = item_index(it, blockIdx.x, gridDim.x);
-      if (idx >= n_items) break;
+    MufuTurn turn;
+    turn.c = &c;
+    turn.slot = s;
+    turn.n = 0;
+    turn.mine = c.bar(B_TOK + 4 * s + warp % 4);
+    turn.theirs = c.bar(B_TOK + 4 * (1 - s) + warp % 4);
+    ItemRing ir{reinterpret_cast<volatile int*>(gbase + OFF_IRING), 0};
+    while (ok) {
+      const int idx = ir.next(c, false);   // every lane reads the entry, then lane 0 releases it
+      __syncwarp();
+      if (lane == 0 && idx >= 0) mbar_arrive(c.bar(B_IEMPTY + ((ir.k - 1) & 1)));
+      if (idx < 0) break;
       const Item I = load_item(items, idx, p, head_mode, H_kv, G);
       if (I.n == 0 || (s == 1 && !I.two)) continue;
+      turn.on = I.two;
+      turn.ok = true;
       const int i = I.T * BM + row;        // query position in the sequence
       const int i_out = I.t * BM + row;    // row of q and o in this call
       const int kind_el = I.kind == EA_STREAMING ? EA_STREAMING : EA_FULL;
@@ -480,15 +567,19 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         uint32_t pk[BN / 2];
         float f;
         if (ct < 0) {
-          f = softmax_tile<1>(x, -1, 0, 0, p.scale_log2, m_ref, l, pk);
+          f = softmax_tile<1>(x, -1, 0, 0, p.scale_log2, m_ref, l, pk, turn);
         } else if (tile_needs_mask(p, I.kind, I.T, ct)) {
           const int lim = i - ct * BN;
           if (kind_el == EA_STREAMING)
-            f = softmax_tile<2>(x, lim, p.n_sink - ct * BN, lim - p.window, p.scale_log2, m_ref, l, pk);
+            f = softmax_tile<2>(x, lim, p.n_sink - ct * BN, lim - p.window, p.scale_log2, m_ref, l, pk, turn);
           else
-            f = softmax_tile<1>(x, lim, 0, 0, p.scale_log2, m_ref, l, pk);
+            f = softmax_tile<1>(x, lim, 0, 0, p.scale_log2, m_ref, l, pk, turn);
         } else {
-          f = softmax_tile<0>(x, 0, 0, 0, p.scale_log2, m_ref, l, pk);
+          f = softmax_tile<0>(x, 0, 0, 0, p.scale_log2, m_ref, l, pk, turn);
+        }
+        if (!__all_sync(0xffffffffu, turn.ok)) {
+          ok = false;
+          break;
         }
         // The previous P_s V product must be done before P_s is rewritten and before O_s
         // (which it accumulates into) is rescaled.
@@ -498,8 +589,7 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           if (!ok) break;
           fence_after_sync();
         }
-        const bool raise = f != 1.f;
-        if (jj > 0 && __any_sync(0xffffffffu, raise)) {   // O (complete up to tile jj-1) *= f
+        if (jj > 0 && __any_sync(0xffffffffu, f != 1.f)) {   // O (complete up to tile jj-1) *= f
 #pragma unroll 1
           for (int q4 = 0; q4 < HD / 32; ++q4) {
             uint32_t r[32];
@@ -549,6 +639,13 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
   fence_before_sync();
   __syncthreads();
+  if (threadIdx.x == 0) {   // the last CTA to finish rewinds the claim counter for the next launch
+    __threadfence();
+    if (atomicAdd(hdr + kWsDone / 4, 1u) == gridDim.x - 1) {
+      atomicExch(hdr + kWsClaim / 4, 0u);
+      atomicExch(hdr + kWsDone / 4, 0u);
+    }
+  }
   if (warp == 1) {
     __syncwarp();
     fence_after_sync();

@@ -33,6 +33,8 @@ constexpr int kTile = 128;
 // Workspace layout of the attention calls (bytes from the workspace base).
 constexpr size_t kWsStatus = 0;        // uint32 sticky status bits
 constexpr size_t kWsNItems = 4;        // uint32 items in the schedule
+constexpr size_t kWsClaim = 8;         // uint32 next item to claim (attention launch)
+constexpr size_t kWsDone = 12;         // uint32 CTAs of the attention launch that finished
 constexpr size_t kWsLivePairs = 16;    // uint64
 constexpr size_t kWsLiveTiles = 24;    // uint64
 constexpr size_t kWsHeader = 256;

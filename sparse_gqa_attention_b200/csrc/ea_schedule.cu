@@ -117,7 +117,11 @@ schedule_kernel(const int* __restrict__ cost, PatternDev p, int H_kv, int G, int
     const int pos = atomicAdd(&bins[item_cost(cost, p.n_qt, H_kv, G, b, h, tl, pr, n_bins)], 1);
     items[pos] = make_int4(b, h, tl, pr);
   }
-  if (tid == 0) hdr[kWsNItems / 4] = (uint32_t)n_items;
+  if (tid == 0) {
+    hdr[kWsNItems / 4] = (uint32_t)n_items;
+    hdr[kWsClaim / 4] = 0u;   // the attention launch claims items from 0
+    hdr[kWsDone / 4] = 0u;
+  }
 }
 
 // grid (n_qt, H_kv, B), 128 threads: thread = query row of tile t.
