@@ -23,6 +23,7 @@
 // and prologue overlap the previous kernel.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstdint>
 #include "ea_common.cuh"
 #include "ea_internal.h"
@@ -99,23 +100,42 @@ pool_partial_kernel(const T* __restrict__ hidden, int S, int D, int n_rows, int 
   }
 }
 
-// hbar[b][c] = (sum over splits of the partial sums) / n_rows, fixed order (ea_router_pool).
+// Sum of the splits sp = first, first + step, ... < n of partial[sp * stride + i], in that
+// order, 8 loads in flight.
+__device__ __forceinline__ float sum_splits(const float* __restrict__ partial, size_t stride, int first, int step,
+                                            int n, size_t i) {
+  float t = 0.f;
+  int sp = first;
+  for (; sp + 7 * step < n; sp += 8 * step) {
+    float y[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) y[u] = partial[(size_t)(sp + u * step) * stride + i];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) t += y[u];
+  }
+  for (; sp < n; sp += step) t += partial[(size_t)sp * stride + i];
+  return t;
+}
+
+// hbar[b][c] = (sum over splits of the partial sums) / n_rows (ea_router_pool).  A CTA takes 32
+// consecutive entries of [B, D]; warp w sums splits w, w+8, ...; the 8 warp sums are added in
+// warp order.
 __global__ void __launch_bounds__(256)
 pool_finish_kernel(const float* __restrict__ partial, int n_splits, int B, int D, float inv_rows,
                    float* __restrict__ hbar) {
+  __shared__ float red[8][32];
   grid_dependency_wait();
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= B * D) return;
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  int sp = 0;
-  for (; sp + 4 <= n_splits; sp += 4) {
-    a0 += partial[(size_t)sp * B * D + i];
-    a1 += partial[(size_t)(sp + 1) * B * D + i];
-    a2 += partial[(size_t)(sp + 2) * B * D + i];
-    a3 += partial[(size_t)(sp + 3) * B * D + i];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const size_t i = (size_t)blockIdx.x * 32 + lane;
+  const bool in = i < (size_t)B * D;
+  red[warp][lane] = in ? sum_splits(partial, (size_t)B * D, warp, 8, n_splits, i) : 0.f;
+  __syncthreads();
+  if (warp == 0 && in) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += red[w][lane];
+    hbar[i] = t * inv_rows;
   }
-  for (; sp < n_splits; ++sp) a0 += partial[(size_t)sp * B * D + i];
-  hbar[i] = ((a0 + a1) + (a2 + a3)) * inv_rows;
 }
 
 constexpr int kProjRows = 32;      // rows of W_k per projection CTA
@@ -145,12 +165,15 @@ __device__ __forceinline__ void fma_vec(float* acc, uint4 raw, float x) {
 //                `partial` is null (boundary pooling), else (sum of the splits' partials) / n_rows
 //   part[n]    = sum_{r in chunk} W_k[r, n] * hbar[b][r]              for every column n < N
 //   pp[cluster][b][n] = sum over the cluster's 8 CTAs of part[n]      (fixed rank order)
+// When its 32 rows of W_k fit (wk_smem), the CTA first copies them into shared memory
+// with asynchronous 16-byte copies, so that the W_k stream overlaps the pooling.
 template <typename T>
 __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kProjThreads)
 project_kernel(const T* __restrict__ hidden, int S, int n_rows, int a_len, int b_start,
                const float* __restrict__ partial, int n_splits, int B, int D, float inv_rows,
-               const T* __restrict__ w_k, int N, int batch, float* __restrict__ pp) {
+               const T* __restrict__ w_k, int N, int batch, float* __restrict__ pp, int wk_smem) {
   constexpr int V = Vec<T>::N;
+  extern __shared__ __align__(16) uint8_t wk_s[];
   constexpr int kColVecs = kProjRows / V;              // 16-byte vectors per pooled row chunk
   constexpr int kTokLanes = kProjThreads / kColVecs;   // token lanes of the fused pooling
   constexpr int kRedRows = kTokLanes > kProjThreads / kProjRows ? kTokLanes : kProjThreads / kProjRows;
@@ -161,10 +184,18 @@ project_kernel(const T* __restrict__ hidden, int S, int n_rows, int a_len, int b
   float (*red)[kProjRows] = reinterpret_cast<float (*)[kProjRows]>(scratch);
   float* accs = scratch;
   launch_dependents();
-  grid_dependency_wait();   // the pooling partial sums (whole-sequence pooling)
   const int r0 = blockIdx.x * kProjRows, tid = threadIdx.x;
   const int rows = max(0, min(kProjRows, D - r0));
   const uint32_t rank = cluster_rank();
+  if (wk_smem) {   // W_k is an input, not the previous kernel's output: copy before waiting
+    const int n16 = rows * N * (int)sizeof(T) / 16;
+    const char* src = reinterpret_cast<const char*>(w_k + (size_t)r0 * N);
+    for (int i = tid; i < n16; i += kProjThreads)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(wk_s + 16 * i)), "l"(src + 16 * i)
+                   : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  grid_dependency_wait();   // the pooling partial sums (whole-sequence pooling)
   const int col_threads = N / V;                          // N % V == 0 (d in {64, 128})
   for (int b0 = 0; b0 < B; b0 += batch) {
     const int nb = min(batch, B - b0);
@@ -199,17 +230,9 @@ project_kernel(const T* __restrict__ hidden, int S, int n_rows, int a_len, int b
       } else {
         // From the splits' partial sums: thread = (row, split lane).
         const int rl = tid % kProjRows, sl = tid / kProjRows, lanes = kProjThreads / kProjRows;
-        float s0 = 0.f, s1 = 0.f;
-        if (rl < rows) {
-          const float* src = partial + (size_t)(b0 + bb) * D + r0 + rl;
-          int sp = sl;
-          for (; sp + lanes < n_splits; sp += 2 * lanes) {
-            s0 += src[(size_t)sp * B * D];
-            s1 += src[(size_t)(sp + lanes) * B * D];
-          }
-          if (sp < n_splits) s0 += src[(size_t)sp * B * D];
-        }
-        red[sl][rl] = s0 + s1;
+        red[sl][rl] = rl < rows ? sum_splits(partial, (size_t)B * D, sl, lanes, n_splits,
+                                             (size_t)(b0 + bb) * D + r0 + rl)
+                                : 0.f;
         __syncthreads();
         if (tid < kProjRows) {
           float t = 0.f;
@@ -219,7 +242,12 @@ project_kernel(const T* __restrict__ hidden, int S, int n_rows, int a_len, int b
         __syncthreads();
       }
     }
+    if (wk_smem && b0 == 0) {
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      __syncthreads();
+    }
     // Partial projections: thread = (column group of V, row lane); columns loop when N/V > threads.
+    const T* wk_base = wk_smem ? reinterpret_cast<const T*>(wk_s) : w_k + (size_t)r0 * N;
     for (int c0 = 0; c0 < col_threads; c0 += kProjThreads) {
       const int cgroups = min(kProjThreads, col_threads - c0);
       const int lanes = max(1, kProjThreads / cgroups);
@@ -230,7 +258,7 @@ project_kernel(const T* __restrict__ hidden, int S, int n_rows, int a_len, int b
 #pragma unroll
         for (int e = 0; e < V; ++e) acc[bb][e] = 0.f;
       if (rl < lanes) {
-        const T* col = w_k + (size_t)r0 * N + (size_t)(c0 + cg) * V;
+        const T* col = wk_base + (size_t)(c0 + cg) * V;
         int r = rl;
         for (; r + 7 * lanes < rows; r += 8 * lanes) {   // 8 loads in flight
           uint4 x[8];
@@ -286,8 +314,6 @@ project_kernel(const T* __restrict__ hidden, int S, int n_rows, int a_len, int b
   }
 }
 
-constexpr int kHeadThreads = 256;  // 8 warps
-constexpr int kHeadWarps = kHeadThreads / 32;
 constexpr int kVC = 16;            // (sample, KV head) vectors per pass through the MLP
 constexpr int kSub = 8;            // vectors per register pass of a warp
 
@@ -337,6 +363,10 @@ __device__ __forceinline__ bool rs_owner(int lane) {   // one lane per replicate
   }
   return own;
 }
+
+// Threads of the router head: 16 warps at head dim 128 (each layer's rows split 4 / 1 / 4 per
+// warp), 8 at head dim 64.
+template <int HD> struct HeadThreads { static constexpr int N = HD == 128 ? 512 : 256; };
 
 // Rows [r0, r0 + RW) of a layer for kSub vectors: acc[r * kSub + v] = W[r] . x_v over K
 // inputs, where x_v = X1[v] (K1 values) followed by X2[v] (K - K1 values).  W: shared
@@ -394,12 +424,13 @@ struct HeadSmem {
 // Layer outputs go to every CTA's shared memory; the final dot product is summed over the
 // CTAs' rows of u in rank order.
 template <int HD>
-__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kHeadThreads, 1)
+__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(HeadThreads<HD>::N, 1)
 router_head_kernel(const float* __restrict__ pp, int n_pp, int BH, int H_kv, const float* __restrict__ w_t1,
                    const float* __restrict__ b_t1, const float* __restrict__ w_t2, const float* __restrict__ b_t2,
                    const float* __restrict__ w_r1, const float* __restrict__ b_r1, const float* __restrict__ w_o,
                    const float* __restrict__ b_o, int32_t* __restrict__ head_mode, float* __restrict__ logits) {
   using L = HeadSmem<HD>;
+  constexpr int kHeadThreads = HeadThreads<HD>::N, kHeadWarps = kHeadThreads / 32;
   extern __shared__ __align__(16) float sm[];
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const uint32_t rank = cluster_rank();
@@ -415,11 +446,14 @@ router_head_kernel(const float* __restrict__ pp, int n_pp, int BH, int H_kv, con
     copy4(sm + L::W1, w_t1 + (size_t)rank * L::R1 * HD, L::R1 * HD);
     copy4(sm + L::W2, w_t2 + (size_t)rank * L::R2 * 4 * HD, L::R2 * 4 * HD);
     copy4(sm + L::W3, w_r1 + (size_t)rank * L::R3 * 2 * HD, L::R3 * 2 * HD);
-    for (int i = tid; i < L::R1; i += kHeadThreads) sm[L::B1 + i] = b_t1[rank * L::R1 + i];
-    for (int i = tid; i < L::R2; i += kHeadThreads) sm[L::B2 + i] = b_t2[rank * L::R2 + i];
-    for (int i = tid; i < L::R3; i += kHeadThreads) sm[L::B3 + i] = b_r1[rank * L::R3 + i];
+    auto copy1 = [&](float* dst, const float* src) {   // 4-byte asynchronous copy
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+    };
+    for (int i = tid; i < L::R1; i += kHeadThreads) copy1(sm + L::B1 + i, b_t1 + rank * L::R1 + i);
+    for (int i = tid; i < L::R2; i += kHeadThreads) copy1(sm + L::B2 + i, b_t2 + rank * L::R2 + i);
+    for (int i = tid; i < L::R3; i += kHeadThreads) copy1(sm + L::B3 + i, b_r1 + rank * L::R3 + i);
     for (int i = tid; i < H_kv * L::R3; i += kHeadThreads)
-      sm[L::WO + i] = w_o[(size_t)(i / L::R3) * 4 * HD + rank * L::R3 + i % L::R3];
+      copy1(sm + L::WO + i, w_o + (size_t)(i / L::R3) * 4 * HD + rank * L::R3 + i % L::R3);
     asm volatile("cp.async.commit_group;" ::: "memory");
   }
   grid_dependency_wait();   // the projection partials
@@ -451,9 +485,10 @@ router_head_kernel(const float* __restrict__ pp, int n_pp, int BH, int H_kv, con
     if (v0 == 0) asm volatile("cp.async.wait_all;" ::: "memory");   // this thread's weight copies
     __syncthreads();
     cluster_sync();
-    // Task MLP hidden layer: this CTA's R1 rows, R1/8 per warp.
+    // Task MLP hidden layer: this CTA's R1 rows, split over the warps.
     for (int s0 = 0; s0 < nv; s0 += kSub) {
-      constexpr int RW = L::R1 / kHeadWarps;
+      constexpr int RW = L::R1 / kHeadWarps > 0 ? L::R1 / kHeadWarps : 1;
+      if (warp * RW >= L::R1) continue;
       float acc[RW * kSub];
       const int ns = min(kSub, nv - s0);
       warp_rows<RW, HD, HD>(sm + L::W1, warp * RW, sm + L::P + s0 * HD, nullptr, ns, lane, acc);
@@ -470,7 +505,8 @@ router_head_kernel(const float* __restrict__ pp, int n_pp, int BH, int H_kv, con
     cluster_sync();
     // Task representation: R2 rows.
     for (int s0 = 0; s0 < nv; s0 += kSub) {
-      constexpr int RW = L::R2 / kHeadWarps;
+      constexpr int RW = L::R2 / kHeadWarps > 0 ? L::R2 / kHeadWarps : 1;
+      if (warp * RW >= L::R2) continue;
       float acc[RW * kSub];
       const int ns = min(kSub, nv - s0);
       warp_rows<RW, 4 * HD, 4 * HD>(sm + L::W2, warp * RW, sm + L::HID + s0 * 4 * HD, nullptr, ns, lane, acc);
@@ -487,7 +523,8 @@ router_head_kernel(const float* __restrict__ pp, int n_pp, int BH, int H_kv, con
     cluster_sync();
     // Router MLP hidden layer on [p; tau]: R3 rows, kept in this CTA.
     for (int s0 = 0; s0 < nv; s0 += kSub) {
-      constexpr int RW = L::R3 / kHeadWarps;
+      constexpr int RW = L::R3 / kHeadWarps > 0 ? L::R3 / kHeadWarps : 1;
+      if (warp * RW >= L::R3) continue;
       float acc[RW * kSub];
       const int ns = min(kSub, nv - s0);
       warp_rows<RW, 2 * HD, HD>(sm + L::W3, warp * RW, sm + L::P + s0 * HD, sm + L::TAU + s0 * HD, ns, lane, acc);
@@ -572,6 +609,19 @@ int proj_batch(int N) { return max(1, min(kProjB, kStageFloats / N)); }
 
 static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+// Raise a kernel's dynamic shared-memory limit once per device (host-side cost off the calls).
+template <auto kern>
+static bool attr_once(int bytes) {
+  static std::atomic<uint64_t> done{0};   // bit per device, one set of bits per kernel
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (done.load() & bit)) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  done.fetch_or(bit);
+  return true;
+}
+
 // Workspace: pooling partial sums [n_splits][B][D] (whole-sequence pooling), then the
 // projection clusters' partials [n_clusters][B][H_kv*d].  The MLP vectors stay in the
 // router head's shared memory.
@@ -595,9 +645,8 @@ static ea_status launch_head(const float* pp, int n_pp, int BH, int H_kv, const 
   auto kern = router_head_kernel<HD>;
   constexpr size_t bytes = HeadSmem<HD>::BYTES;
   static_assert(bytes <= 232448, "router head shared memory beyond the 227 KB a CTA may use");
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
-    return EA_ERR_CUDA;
-  return launch_after(kern, dim3(kCluster), dim3(kHeadThreads), bytes, st, true, pp, n_pp, BH, H_kv, w->w_t1,
+  if (!attr_once<router_head_kernel<HD>>((int)bytes)) return EA_ERR_CUDA;
+  return launch_after(kern, dim3(kCluster), dim3(HeadThreads<HD>::N), bytes, st, true, pp, n_pp, BH, H_kv, w->w_t1,
                       w->b_t1, w->w_t2, w->b_t2, w->w_r1, w->b_r1, w->w_o, w->b_o, head_mode, logits) == cudaSuccess
              ? EA_OK
              : EA_ERR_CUDA;
@@ -615,9 +664,14 @@ static ea_status launch_pool_project(const T* hidden, int B, int S, int D, int N
                                                          pl.rows_per_split, partial);
     if (cudaGetLastError() != cudaSuccess) return EA_ERR_CUDA;
   }
-  const cudaError_t e = launch_after(project_kernel<T>, dim3(proj_ctas(D)), dim3(kProjThreads), 0, st, !fused,
+  // W_k rows staged in shared memory when they fit next to the static buffers.
+  const size_t wk_bytes = (size_t)kProjRows * N * sizeof(T);
+  const int wk_smem = wk_bytes <= 96 * 1024 && (N * sizeof(T)) % 16 == 0 ? 1 : 0;
+  const size_t dyn = wk_smem ? wk_bytes : 0;
+  if (!attr_once<project_kernel<T>>(96 * 1024)) return EA_ERR_CUDA;
+  const cudaError_t e = launch_after(project_kernel<T>, dim3(proj_ctas(D)), dim3(kProjThreads), dyn, st, !fused,
                                      hidden, S, pl.n_rows, pl.a_len, pl.b_start, fused ? nullptr : partial,
-                                     pl.n_splits, B, D, 1.0f / (float)pl.n_rows, w_k, N, proj_batch(N), pp);
+                                     pl.n_splits, B, D, 1.0f / (float)pl.n_rows, w_k, N, proj_batch(N), pp, wk_smem);
   return e == cudaSuccess ? EA_OK : EA_ERR_CUDA;
 }
 
@@ -651,7 +705,7 @@ ea_status launch_router_pool(const void* hidden, ea_dtype dtype, int B, int S, i
     pool_partial_kernel<float><<<g1, kPoolThreads, 0, st>>>(static_cast<const float*>(hidden), S, D, pl.n_rows,
                                                              pl.a_len, pl.b_start, pl.rows_per_split, partial);
   if (cudaGetLastError() != cudaSuccess) return EA_ERR_CUDA;
-  return launch_after(pool_finish_kernel, dim3(cdiv(B * D, 256)), dim3(256), 0, st, true, partial, pl.n_splits, B, D,
+  return launch_after(pool_finish_kernel, dim3(cdiv(B * D, 32)), dim3(256), 0, st, true, partial, pl.n_splits, B, D,
                       1.0f / (float)pl.n_rows, hbar) == cudaSuccess
              ? EA_OK
              : EA_ERR_CUDA;
