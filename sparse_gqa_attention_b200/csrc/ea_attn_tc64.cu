@@ -1,10 +1,10 @@
 // ea_attn_tc64.cu — the hybrid-head attention kernel for block-64 layouts (the pages'
 // block edge: "Elastic Attention: Test-time Adaptive Sparsity Ratios for Efficient
 // Transformers", appendix D.1 "Sparse Inference", block size 64).
-//
-// Same design and pipeline as ea_attn_tc.cu (read its header for the warp roles, TMEM
-// and shared-memory layout, and the bounded waits); the differences are the tile walk
-// and the masking.  Tiles stay 128 x 128; each holds 2 x 2 blocks of 64:
+// Same design and pipeline as ea_attn_tc.cu (read its header for the warp roles, TMEM and
+// shared-memory layout, the MUFU turns, run-time item claims and bounded waits; the shared
+// pieces are in ea_attn_tc.cuh); the differences are the tile walk and the masking.
+// Tiles stay 128 x 128; each holds 2 x 2 blocks of 64:
 //   block-sparse heads   the live key tiles of query tile t are the union of the key
 //                        blocks listed for query blocks 2t and 2t+1 (block kb lies in tile
 //                        kb/2); each tile carries the 2x2 map of its live blocks;
@@ -14,120 +14,15 @@
 // diagonal) the softmax applies the causal rule within the 64-key halves its query
 // half may read.  It is a separate kernel (not a template parameter of the block-128
 // one) so that the block-128 kernel keeps its measured code.
-#include <cuda.h>
-#include <cuda_bf16.h>
-#include <cuda_runtime.h>
-#include <cstdint>
-#include <mutex>
-#include "ea_common.cuh"
+#include <atomic>
+#include "ea_attn_tc.cuh"
 #include "ea_internal.h"
-#include "ea_sm100.cuh"
 
 namespace ea {
+
 namespace {
 
-using namespace sm100;
-
-constexpr int BM = 128, BN = 128, HD = 128;
-constexpr int NKV = 3;                                 // K/V ring slots
-constexpr int kThreads = 384;
-constexpr uint32_t kTileBytes = BM * HD * 2;           // 32 KB per 128x128 bf16 tile
-constexpr uint32_t kBoxBytes = kTileBytes / 2;         // one 64-column box
-constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_P = 2 * kTileBytes;
-constexpr uint32_t OFF_KV = 4 * kTileBytes;
-constexpr uint32_t OFF_BAR = OFF_KV + NKV * kTileBytes;
-enum : int {
-  B_QFULL = 0, B_QEMPTY = 2, B_KVFULL = 4, B_KVEMPTY = B_KVFULL + NKV, B_SFULL = B_KVEMPTY + NKV,
-  B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2, B_PVDONE = B_PFULL + 2, B_OFULL = B_PVDONE + 2,
-  B_FIN = B_OFULL + 2, B_NEVER = B_FIN + 1, N_BAR = B_NEVER + 1
-};
-constexpr uint32_t OFF_TMEM = OFF_BAR + N_BAR * 8;
-constexpr uint32_t OFF_ABORT = OFF_TMEM + 4;
-constexpr uint32_t kSmemBytes = OFF_ABORT + 4 + 1024;  // + slack to align the base to 1024
-static_assert(kSmemBytes <= 232448, "shared memory beyond the 227 KB a CTA may use");
-constexpr uint32_t kTmemCols = 512;
-__device__ __forceinline__ uint32_t col_s(int s) { return 128u * s; }        // S_s (and P_s) columns
-__device__ __forceinline__ uint32_t col_o(int s) { return 256u + 128u * s; } // O_s columns
-constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, false);
-constexpr uint32_t IDESC_PV = idesc_bf16(BM, HD, true);
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
-constexpr float kRescaleLog2 = 8.0f;
-
-// Register split: the launch gives 384 x 168 = 64512 registers; warpgroup 0 (producer,
-// MMA, two idle warps) drops to 88 and the two softmax warpgroups rise to 208:
-// 128 x 88 + 256 x 208 = 64512.
-constexpr int kRegsCtl = 88, kRegsSoftmax = 208;
-static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= kThreads * 168, "register split exceeds the launch");
-
-struct Ctx {
-  uint32_t bar0;                 // shared address of barrier 0
-  volatile int* abort_flag;
-  uint32_t* status;
-  __device__ uint32_t bar(int i) const { return bar0 + 8u * i; }
-};
-
-__device__ __forceinline__ bool wait_slow(const Ctx& c, uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (*c.abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      *c.abort_flag = 1;
-      atomicOr(c.status, kStatusTimeout);
-      return false;
-    }
-  }
-  return true;
-}
-__device__ __forceinline__ bool wait(const Ctx& c, uint32_t bar, uint32_t parity) {
-  return mbar_try_wait(bar, parity) || wait_slow(c, bar, parity);
-}
-// Drain wait: also after an abort, wait (bounded) for this CTA's own copies and MMAs.
-__device__ __forceinline__ void wait_drain(const Ctx& c, uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      atomicOr(c.status, kStatusTimeout);
-      return;
-    }
-  }
-}
-
-struct Item {
-  int b, h, t, T, pr, kind, n, sink_end, win_lo;   // t: query tile of this call, T: of the sequence
-  long long csr_beg;
-  bool two;
-};
-
-__device__ __forceinline__ int item_index(int it, int cta, int ncta) {
-  return it * ncta + ((it & 1) ? (ncta - 1 - cta) : cta);
-}
-
-__device__ __forceinline__ Item load_item(const int4* items, int idx, const PatternDev& p,
-                                          const int32_t* head_mode, int H_kv, int G) {
-  const int4 w = items[idx];
-  Item I;
-  I.b = w.x; I.h = w.y; I.t = w.z; I.pr = w.w;
-  I.T = I.t + p.q_tile0;
-  I.kind = head_kind(p, head_mode, H_kv, I.b, I.h);
-  I.two = 2 * I.pr + 1 < G;
-  I.sink_end = I.win_lo = 0;
-  I.csr_beg = 0;
-  if (is_streaming(I.kind)) {
-    stream_ranges(p, I.kind, I.T, I.sink_end, I.win_lo);
-    I.n = I.sink_end + max(0, I.T - I.win_lo + 1);
-  } else if (bs64_kind(p, I.kind)) {
-    I.n = n_live_tiles(p, I.kind, H_kv, I.b, I.h, I.T);
-  } else if (I.kind == EA_BLOCK_SPARSE) {
-    long long a, e;
-    csr_row(p, H_kv, I.b, I.h, I.T, a, e);
-    I.csr_beg = a;
-    I.n = (int)(e - a);
-  } else {
-    I.n = I.T + 1;
-  }
-  return I;
-}
+using namespace tc;
 
 // Sequential walk over an item's live key tiles: the tile index (-1: nothing live) and,
 // for block-64 block-sparse heads, the 2x2 map of its live blocks (0xF otherwise).
@@ -155,120 +50,11 @@ __device__ __forceinline__ Walk start_walk(const PatternDev& p, const Item& I, i
   return k;
 }
 
-__device__ __forceinline__ uint64_t qk_desc(uint32_t tile, int kk) {
-  // K-major operand: rows of 128 bytes, 8-row swizzle atoms 1024 bytes apart (SBO);
-  // K step kk of 16 elements = +32 bytes inside a 64-column box, boxes 16 KB apart.
-  return sdesc_sw128(tile + (uint32_t)(kk >> 2) * kBoxBytes + (uint32_t)(kk & 3) * 32u, 16u, 1024u);
-}
-__device__ __forceinline__ uint64_t v_desc(uint32_t tile, int kk) {
-  // MN-major operand (N = head dim, contiguous): 64-column boxes 16 KB apart (LBO),
-  // 8-key groups 1024 bytes apart (SBO); K step kk of 16 keys = +2048 bytes.
-  return sdesc_sw128(tile + (uint32_t)kk * 2048u, kBoxBytes, 1024u);
-}
-
-// S_s = Q_s K^T for the key tile at kt, once the softmax has loaded the previous S_s.
-__device__ __forceinline__ bool issue_qk(const Ctx& c, uint32_t tmem, uint32_t base, int s, uint32_t kt,
-                                         int& s_cnt) {
-  if (s_cnt > 0 && !wait(c, c.bar(B_SFREE + s), (s_cnt - 1) & 1)) return false;
-  fence_after_sync();
-  const uint32_t qt = base + OFF_Q + s * kTileBytes;
-#pragma unroll
-  for (int kk = 0; kk < HD / 16; ++kk)
-    mma_ss(tmem + col_s(s), qk_desc(qt, kk), qk_desc(kt, kk), IDESC_QK, kk > 0 ? 1u : 0u);
-  commit(c.bar(B_SFULL + s));
-  ++s_cnt;
-  return true;
-}
-
-// O_s (+)= P_s V for the V tile at vt, once the softmax has written P_s.
-__device__ __forceinline__ bool issue_pv(const Ctx& c, uint32_t tmem, uint32_t base, int s, uint32_t vt,
-                                         bool accumulate, bool last, int& p_cnt) {
-  if (!wait(c, c.bar(B_PFULL + s), p_cnt & 1)) return false;
-  ++p_cnt;
-  fence_after_sync();
-  const uint32_t pt = base + OFF_P + s * kTileBytes;
-#pragma unroll
-  for (int kk = 0; kk < BN / 16; ++kk)
-    mma_ss(tmem + col_o(s), qk_desc(pt, kk), v_desc(vt, kk), IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
-  commit(c.bar(B_PVDONE + s));
-  if (last) {
-    commit(c.bar(B_OFULL + s));
-    commit(c.bar(B_QEMPTY + s));
-  }
-  return true;
-}
-
-// One 128-key tile of one query row: running max (raised only past kRescaleLog2),
-// row sum, and P = exp2(scale*log2e*s - max) as bf16 pairs in pk (pk[j] holds keys
-// 2j, 2j+1).  kMode 0: every key live; 1: causal rule; 2: streaming rule; 3: causal
-// rule within the enabled 64-key halves (block-64 kinds; sink_lim holds the bits).  Returns
-// the factor O must be multiplied by (1 when the max was not raised).
-template <int kMode>
-__device__ __forceinline__ float softmax_tile(const float (&x)[BN], int lim, int sink_lim, int win_lim,
-                                              float scale_log2, float& m_ref, float& l, uint32_t (&pk)[BN / 2]) {
-  auto live = [&](int e) {
-    if (kMode == 0) return true;
-    if (kMode == 1) return e <= lim;
-    if (kMode == 3) return e <= lim && ((sink_lim >> (e >> 6)) & 1) != 0;   // sink_lim: key-half bits
-    return e <= lim && (e < sink_lim || e > win_lim);
-  };
-  auto xm = [&](int e) { return live(e) ? x[e] : -INFINITY; };
-  // Row max as 8 independent 3-input chains over 16 columns each, then a short tree.
-  float m8[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    m8[c] = xm(16 * c);
-#pragma unroll
-    for (int e = 1; e + 1 < 16; e += 2) m8[c] = fmax3(m8[c], xm(16 * c + e), xm(16 * c + e + 1));
-    m8[c] = fmaxf(m8[c], xm(16 * c + 15));
-  }
-  const float mt = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
-  const float mts = mt * scale_log2;
-  float f = 1.f;
-  if (mts > m_ref + kRescaleLog2) {
-    f = ex2(m_ref - mts);  // 0 while m_ref is still -inf
-    l *= f;
-    m_ref = mts;
-  }
-  const float sub = (m_ref == -INFINITY) ? 0.f : m_ref;
-  const uint64_t scale2 = f2_pack(scale_log2, scale_log2), nsub2 = f2_pack(-sub, -sub);
-  uint64_t l2 = f2_pack(0.f, 0.f);
-#pragma unroll
-  for (int e = 0; e < BN; e += 2) {
-    float t0, t1;
-    f2_unpack(f2_fma(f2_pack(x[e], x[e + 1]), scale2, nsub2), t0, t1);
-    const float p0 = live(e) ? ex2(t0) : 0.f;
-    const float p1 = live(e + 1) ? ex2(t1) : 0.f;
-    l2 = f2_add(l2, f2_pack(p0, p1));
-    pk[e / 2] = pack_bf16x2(p0, p1);
-  }
-  float la, lb;
-  f2_unpack(l2, la, lb);
-  l += la + lb;
-  return f;
-}
-
-// Row `row` of P into the K-major, 128-byte-swizzled tile at p_tile: keys 64b..64b+63
-// in box b, 16-byte chunk c of a row at chunk position c ^ (row % 8).
-__device__ __forceinline__ void store_p_row(uint32_t p_tile, int row, const uint32_t (&pk)[BN / 2]) {
-#pragma unroll
-  for (int bx = 0; bx < 2; ++bx) {
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-      const uint32_t addr = p_tile + bx * kBoxBytes + (uint32_t)row * 128u + (uint32_t)((ch ^ (row & 7)) << 4);
-      const int j = 32 * bx + 4 * ch;
-      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[j]), "r"(pk[j + 1]),
-                   "r"(pk[j + 2]), "r"(pk[j + 3])
-                   : "memory");
-    }
-  }
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
 hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o,
                       const int32_t* __restrict__ head_mode, const PatternDev p, int S, int H_q, int H_kv,
-                      const int4* __restrict__ items, uint32_t* __restrict__ hdr) {
+                      const int4* __restrict__ items, uint32_t* __restrict__ hdr, int inject_stall) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -287,7 +73,9 @@ hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     tma_prefetch_map(&tm_v);
     for (int i = 0; i < N_BAR; ++i) {
       const bool softmax_arrive = (i >= B_SFREE && i < B_SFREE + 2) || (i >= B_PFULL && i < B_PFULL + 2);
-      mbar_init(c.bar(i), softmax_arrive ? 128u : 1u);
+      const bool token = i >= B_TOK && i < B_TOK + 8;   // one softmax warp arrives
+      const bool item_read = i >= B_IEMPTY && i < B_IEMPTY + 2;
+      mbar_init(c.bar(i), softmax_arrive ? 128u : token ? 32u : item_read ? kItemReaders : 1u);
     }
     *c.abort_flag = 0;
     fence_mbar_init();
@@ -318,10 +106,18 @@ hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         ++kv;
         return true;
       };
+      volatile int* ring = reinterpret_cast<volatile int*>(gbase + OFF_IRING);
       for (int it = 0; ok; ++it) {
-        const int idx = item_index(it, blockIdx.x, gridDim.x);
-        if (idx >= n_items) break;
-        const Item I = load_item(items, idx, p, head_mode, H_kv, G);
+        // Claim the next item once the readers are done with this ring entry's last use.
+        const int e = it & 1;
+        ok = wait(c, c.bar(B_IEMPTY + e), ((it >> 1) & 1) ^ 1);
+        if (!ok) break;
+        int idx = (int)atomicAdd(hdr + kWsClaim / 4, 1u);
+        if (idx >= n_items) idx = -1;
+        ring[e] = idx;
+        mbar_arrive(c.bar(B_IFULL + e));
+        if (idx < 0) break;
+        const Item I = load_item<true>(items, idx, p, head_mode, H_kv, G);
         if (I.n == 0) continue;
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
@@ -355,15 +151,30 @@ hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         if (q_use[s] > 0) wait_drain(c, c.bar(B_QFULL + s), (q_use[s] - 1) & 1);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ Q K^T issuer
+    // Walks the ring in the producer's order; takes the K entries, skips the V entries.
     if (lane == 0) {
-      int q_use[2] = {0, 0}, s_cnt[2] = {0, 0}, p_cnt[2] = {0, 0};
+      int q_use[2] = {0, 0}, s_cnt[2] = {0, 0};
       int kv = 0;
-      bool ok = true;
-      for (int it = 0; ok; ++it) {
-        const int idx = item_index(it, blockIdx.x, gridDim.x);
-        if (idx >= n_items) break;
-        const Item I = load_item(items, idx, p, head_mode, H_kv, G);
+      // Test hook for the timeout path: CTA 0 first waits on a barrier nothing arrives on.
+      bool ok = !(inject_stall && blockIdx.x == 0) || wait(c, c.bar(B_NEVER), 0);
+      // S of key tile jj (both slots); the ring slot is released once both products finish.
+      auto qk_tile = [&](const Item& I, int jj) -> bool {
+        const int slot = kv % NKV;
+        if (!wait(c, c.bar(B_KVFULL + slot), (kv / NKV) & 1)) return false;
+        const uint32_t kt = base + OFF_KV + slot * kTileBytes;
+        const bool last = jj + 1 == I.n;
+        if (!issue_qk(c, tmem, base, 0, kt, s_cnt[0], last)) return false;
+        if (I.two && !issue_qk(c, tmem, base, 1, kt, s_cnt[1], last)) return false;
+        commit(c.bar(B_KVEMPTY + slot));
+        ++kv;
+        return true;
+      };
+      ItemRing ir{reinterpret_cast<volatile int*>(gbase + OFF_IRING), 0};
+      while (ok) {
+        const int idx = ir.next(c, true);
+        if (idx < 0) break;
+        const Item I = load_item<true>(items, idx, p, head_mode, H_kv, G);
         if (I.n == 0) continue;
         ok = wait(c, c.bar(B_QFULL + 0), q_use[0] & 1);
         ++q_use[0];
@@ -371,35 +182,36 @@ hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           ok = ok && wait(c, c.bar(B_QFULL + 1), q_use[1] & 1);
           ++q_use[1];
         }
-        // S of the item's first key tile; the ring slot is released once both products finish.
-        {
-          const int slot = kv % NKV;
-          ok = ok && wait(c, c.bar(B_KVFULL + slot), (kv / NKV) & 1);
-          if (ok) {
-            const uint32_t kt = base + OFF_KV + slot * kTileBytes;
-            ok = issue_qk(c, tmem, base, 0, kt, s_cnt[0]);
-            if (ok && I.two) ok = issue_qk(c, tmem, base, 1, kt, s_cnt[1]);
-            if (ok) commit(c.bar(B_KVEMPTY + slot));
-            ++kv;
-          }
-        }
+        ok = ok && qk_tile(I, 0);
         for (int jj = 0; jj < I.n && ok; ++jj) {
-          const bool last = jj + 1 == I.n;
-          if (!last) {   // the next scores first: they run while the softmax works on tile jj
-            const int slot = kv % NKV;
-            ok = wait(c, c.bar(B_KVFULL + slot), (kv / NKV) & 1);
-            if (!ok) break;
-            const uint32_t kt = base + OFF_KV + slot * kTileBytes;
-            ok = issue_qk(c, tmem, base, 0, kt, s_cnt[0]);
-            if (ok && I.two) ok = issue_qk(c, tmem, base, 1, kt, s_cnt[1]);
-            if (!ok) break;
-            commit(c.bar(B_KVEMPTY + slot));
-            ++kv;
-          }
+          if (jj + 1 < I.n) ok = qk_tile(I, jj + 1);   // ring order: K(jj+1), then V(jj)
+          ++kv;                                       // V(jj): the P V issuer's entry
+        }
+      }
+      commit(c.bar(B_FIN));                       // every MMA issued here has completed
+      wait_drain(c, c.bar(B_FIN), 0);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ P V issuer
+    // Walks the ring in the producer's order; takes the V entries, skips the K entries.
+    if (lane == 0) {
+      int p_cnt[2] = {0, 0};
+      int kv = 0;
+      bool ok = true;
+      ItemRing ir{reinterpret_cast<volatile int*>(gbase + OFF_IRING), 0};
+      while (ok) {
+        const int idx = ir.next(c, true);
+        if (idx < 0) break;
+        const Item I = load_item<true>(items, idx, p, head_mode, H_kv, G);
+        if (I.n == 0) continue;
+        ++kv;                                         // K(0)
+        for (int jj = 0; jj < I.n && ok; ++jj) {
+          if (jj + 1 < I.n) ++kv;                     // K(jj+1)
           const int slot = kv % NKV;
           ok = wait(c, c.bar(B_KVFULL + slot), (kv / NKV) & 1);
           if (!ok) break;
           const uint32_t vt = base + OFF_KV + slot * kTileBytes;
+          const bool last = jj + 1 == I.n;
           ok = issue_pv(c, tmem, base, 0, vt, jj > 0, last, p_cnt[0]);
           if (ok && I.two) ok = issue_pv(c, tmem, base, 1, vt, jj > 0, last, p_cnt[1]);
           if (!ok) break;
@@ -407,8 +219,8 @@ hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           ++kv;
         }
       }
-      commit(c.bar(B_FIN));                       // every MMA issued here has completed
-      wait_drain(c, c.bar(B_FIN), 0);
+      commit(c.bar(B_FIN2));
+      wait_drain(c, c.bar(B_FIN2), 0);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax slots
@@ -419,17 +231,28 @@ hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     const uint32_t p_tile = base + OFF_P + s * kTileBytes;
     int s_cnt = 0, p_cnt = 0, o_cnt = 0;
     bool ok = true;
-    for (int it = 0; ok; ++it) {
-      const int idx = item_index(it, blockIdx.x, gridDim.x);
-      if (idx >= n_items) break;
-      const Item I = load_item(items, idx, p, head_mode, H_kv, G);
+    MufuTurn turn;
+    turn.c = &c;
+    turn.slot = s;
+    turn.n = 0;
+    turn.mine = c.bar(B_TOK + 4 * s + warp % 4);
+    turn.theirs = c.bar(B_TOK + 4 * (1 - s) + warp % 4);
+    ItemRing ir{reinterpret_cast<volatile int*>(gbase + OFF_IRING), 0};
+    while (ok) {
+      const int idx = ir.next(c, false);   // every lane reads the entry, then lane 0 releases it
+      __syncwarp();
+      if (lane == 0 && idx >= 0) mbar_arrive(c.bar(B_IEMPTY + ((ir.k - 1) & 1)));
+      if (idx < 0) break;
+      const Item I = load_item<true>(items, idx, p, head_mode, H_kv, G);
       if (I.n == 0 || (s == 1 && !I.two)) continue;
+      turn.on = I.two;
+      turn.ok = true;
       const int i = I.T * BM + row;        // query position in the sequence
       const int i_out = I.t * BM + row;    // row of q and o in this call
       const int kind_el = I.kind == EA_STREAMING ? EA_STREAMING : EA_FULL;
-      float m_ref = -INFINITY, l = 0.f;
       const bool blk64 = p.block == 64 && (I.kind == EA_BLOCK_SPARSE || I.kind == EA_STREAMING_BLOCKS);
       Walk walk = start_walk(p, I, H_kv);
+      float m_ref = -INFINITY, l = 0.f;
       for (int jj = 0; jj < I.n; ++jj) {
         uint32_t map;
         const int ct = walk.next(p, I, map);
@@ -454,21 +277,25 @@ hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         uint32_t pk[BN / 2];
         float f;
         if (ct < 0) {
-          f = softmax_tile<1>(x, -1, 0, 0, p.scale_log2, m_ref, l, pk);
+          f = softmax_tile<1>(x, -1, 0, 0, p.scale_log2, m_ref, l, pk, turn);
         } else if (blk64) {   // 64x64 blocks: the key halves this warp's query half may read
           const int hb = (int)half_bits(p, I.kind, I.T, ct, row >> 6, map);
           if (hb == 3 && ct < I.T)
-            f = softmax_tile<0>(x, 0, 0, 0, p.scale_log2, m_ref, l, pk);
+            f = softmax_tile<0>(x, 0, 0, 0, p.scale_log2, m_ref, l, pk, turn);
           else
-            f = softmax_tile<3>(x, i - ct * BN, hb, 0, p.scale_log2, m_ref, l, pk);
+            f = softmax_tile<3>(x, i - ct * BN, hb, 0, p.scale_log2, m_ref, l, pk, turn);
         } else if (tile_needs_mask(p, I.kind, I.T, ct)) {
           const int lim = i - ct * BN;
           if (kind_el == EA_STREAMING)
-            f = softmax_tile<2>(x, lim, p.n_sink - ct * BN, lim - p.window, p.scale_log2, m_ref, l, pk);
+            f = softmax_tile<2>(x, lim, p.n_sink - ct * BN, lim - p.window, p.scale_log2, m_ref, l, pk, turn);
           else
-            f = softmax_tile<1>(x, lim, 0, 0, p.scale_log2, m_ref, l, pk);
+            f = softmax_tile<1>(x, lim, 0, 0, p.scale_log2, m_ref, l, pk, turn);
         } else {
-          f = softmax_tile<0>(x, 0, 0, 0, p.scale_log2, m_ref, l, pk);
+          f = softmax_tile<0>(x, 0, 0, 0, p.scale_log2, m_ref, l, pk, turn);
+        }
+        if (!__all_sync(0xffffffffu, turn.ok)) {
+          ok = false;
+          break;
         }
         // The previous P_s V product must be done before P_s is rewritten and before O_s
         // (which it accumulates into) is rescaled.
@@ -478,8 +305,7 @@ hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           if (!ok) break;
           fence_after_sync();
         }
-        const bool raise = f != 1.f;
-        if (jj > 0 && __any_sync(0xffffffffu, raise)) {   // O (complete up to tile jj-1) *= f
+        if (jj > 0 && __any_sync(0xffffffffu, f != 1.f)) {   // O (complete up to tile jj-1) *= f
 #pragma unroll 1
           for (int q4 = 0; q4 < HD / 32; ++q4) {
             uint32_t r[32];
@@ -529,49 +355,18 @@ hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
 
   fence_before_sync();
   __syncthreads();
+  if (threadIdx.x == 0) {   // the last CTA to finish rewinds the claim counter for the next launch
+    __threadfence();
+    if (atomicAdd(hdr + kWsDone / 4, 1u) == gridDim.x - 1) {
+      atomicExch(hdr + kWsClaim / 4, 0u);
+      atomicExch(hdr + kWsDone / 4, 0u);
+    }
+  }
   if (warp == 1) {
     __syncwarp();
     fence_after_sync();
     tmem_dealloc(tmem, kTmemCols);
   }
-}
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  });
-  return fn;
-}
-
-// [B, S, H, 128] bf16 viewed as 4-D (d, H, S, B); box = 64 columns x 1 head x 128 rows.
-bool make_map(CUtensorMap* m, const void* ptr, int B, int S, int H) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[4] = {(cuuint64_t)HD, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
-  const cuuint64_t strides[3] = {(cuuint64_t)HD * 2, (cuuint64_t)H * HD * 2, (cuuint64_t)S * H * HD * 2};
-  const cuuint32_t box[4] = {64, 1, (cuuint32_t)BM, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
-  return n;
 }
 
 }  // namespace
@@ -589,9 +384,10 @@ ea_status launch_attn_tc64(const void* q, const void* k, const void* v, void* o,
     return EA_ERR_CUDA;
   char* ws = static_cast<char*>(workspace);
   const size_t items_off = kWsHeader + ((size_t)B * 4 + 255) / 256 * 256;
+  const int inject = take_inject_stall() ? 1 : 0;
   kern<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), head_mode, pat, S, H_q,
                                            H_kv, reinterpret_cast<const int4*>(ws + items_off),
-                                           reinterpret_cast<uint32_t*>(ws));
+                                           reinterpret_cast<uint32_t*>(ws), inject);
   return cudaGetLastError() == cudaSuccess ? EA_OK : EA_ERR_CUDA;
 }
 

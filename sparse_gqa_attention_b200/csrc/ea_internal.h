@@ -30,6 +30,9 @@ ea_status launch_attn_simt(const float* q, const float* k, const float* v, float
 ea_status launch_attn_tc(const void* q, const void* k, const void* v, void* o, const int32_t* head_mode,
                          const PatternDev& pat, int B, int S, int S_k, int H_q, int H_kv, void* workspace,
                          cudaStream_t st);
+// Test hook (ea_debug_inject_stall): true for the next N launches of a kernel with bounded
+// pipeline waits; that launch's first CTA then waits on a barrier nothing arrives on.
+bool take_inject_stall();
 // Block-64 layouts (ea_attn_tc64.cu); launch_attn_tc forwards to it.
 ea_status launch_attn_tc64(const void* q, const void* k, const void* v, void* o, const int32_t* head_mode,
                            const PatternDev& pat, int B, int S, int S_k, int H_q, int H_kv, void* workspace,

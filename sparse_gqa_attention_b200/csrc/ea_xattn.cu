@@ -47,7 +47,7 @@ constexpr uint32_t X_OFF_A = 0;
 constexpr uint32_t X_OFF_B = XNS * kChunkBytes;
 constexpr uint32_t X_OFF_BAR = XNS * (kChunkBytes + kBChunkBytes);
 enum : int { X_FULL = 0, X_EMPTY = XNS, X_AFULL = 2 * XNS, X_AEMPTY = X_AFULL + 2, X_FIN = X_AEMPTY + 2,
-             X_NBAR = X_FIN + 1 };
+             X_NEVER = X_FIN + 1, X_NBAR = X_NEVER + 1 };
 constexpr uint32_t X_OFF_TMEM = X_OFF_BAR + X_NBAR * 8;
 constexpr uint32_t X_OFF_ABORT = X_OFF_TMEM + 4;
 constexpr uint32_t kXSmemBytes = X_OFF_ABORT + 4 + 1024;   // + slack to align the base to 1024
@@ -201,7 +201,8 @@ template <int ST, int NB>
 __global__ void __launch_bounds__(kXThreads, 1)
 xattn_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, int H_q,
                    int H_kv, int n_red, int n_rt, float sl2, const int* __restrict__ plan,
-                   uint32_t* __restrict__ hdr, float* __restrict__ m_part, float* __restrict__ s_part) {
+                   uint32_t* __restrict__ hdr, float* __restrict__ m_part, float* __restrict__ s_part,
+                   int inject_stall) {
   constexpr int NCH = 2 * ST;   // K chunks per tile: ST row offsets x two 64-column halves of d
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -263,7 +264,8 @@ xattn_score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       int ch = 0, tile = 0;
-      bool ok = true;
+      // Test hook for the timeout path: CTA 0 first waits on a barrier nothing arrives on.
+      bool ok = !(inject_stall && blockIdx.x == 0) || xwait(c, c.bar(X_NEVER), 0);
       for (int it = 0; ok; ++it) {
         const int idx = x_item_index(it, blockIdx.x, gridDim.x);
         if (idx >= n_work) break;
@@ -635,7 +637,9 @@ ea_status launch_st(const void* q, const void* k, const int32_t* head_mode, cons
     return EA_ERR_CUDA;
   const long long max_work = (long long)B * H_q * L.n_rt;
   const int grid = (int)std::min<long long>(max_work, x_sm_count());
-  kern<<<grid, kXThreads, kXSmemBytes, st>>>(mq, mk, H_q, H_kv, L.n_red, L.n_rt, sl2, plan, hdr, m_part, s_part);
+  const int inject = take_inject_stall() ? 1 : 0;
+  kern<<<grid, kXThreads, kXSmemBytes, st>>>(mq, mk, H_q, H_kv, L.n_red, L.n_rt, sl2, plan, hdr, m_part, s_part,
+                                             inject);
   if (cudaGetLastError() != cudaSuccess) return EA_ERR_CUDA;
   dim3 sgrid(L.n_qb, H_kv, B);
   xattn_select_kernel<ST, NB><<<sgrid, kSelThreads, 0, st>>>(head_mode, pd, H_q, H_kv, L.n_red, L.n_rt, tau, m_part,
