@@ -281,6 +281,118 @@ __device__ __forceinline__ float softmax_tile(const float (&x)[BN], int lim, int
   return f;
 }
 
+// softmax_tile for the block-64 kinds' tiles (kMode 3 mostly): the same results, with the
+// masks applied per 32-key chunk with a decision that is the same for the whole
+// warp: a chunk dead for every lane is skipped (no exponentials), one live for every lane
+// runs without per-key tests, and only a mixed chunk tests each key (it computes every
+// exponential and selects, so the MUFU stays pipelined; per-key branches around the
+// exponentials would serialise them).  The exponentials run inside this warp's MUFU turn
+// (tok).  Returns the factor O must be multiplied by (1 when the max was not raised).
+template <int kMode, typename Tok>
+__device__ __forceinline__ float softmax_tile_chunked(const float (&x)[BN], int lim, int sink_lim, int win_lim,
+                                              float scale_log2, float& m_ref, float& l, uint32_t (&pk)[BN / 2],
+                                              Tok& tok) {
+  auto live = [&](int e) {
+    if (kMode == 0) return true;
+    if (kMode == 1) return e <= lim;
+    if (kMode == 3) return e <= lim && ((sink_lim >> (e >> 6)) & 1) != 0;   // sink_lim: key-half bits
+    return e <= lim && (e < sink_lim || e > win_lim);
+  };
+  // Chunk classes (0 dead, 1 live, 2 mixed) from the warp's extremes of the per-lane limits.
+  int cls[4] = {1, 1, 1, 1};
+  if (kMode != 0) {
+    const int lo = __reduce_min_sync(0xffffffffu, lim), hi = __reduce_max_sync(0xffffffffu, lim);
+    int wlo = 0, whi = 0;
+    if (kMode == 2) {
+      wlo = __reduce_min_sync(0xffffffffu, win_lim);
+      whi = __reduce_max_sync(0xffffffffu, win_lim);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int a = 32 * c, b = a + 31;
+      int k = a > hi ? 0 : (b <= lo ? 1 : 2);                     // causal part
+      if (kMode == 3 && ((sink_lim >> (a >> 6)) & 1) == 0) k = 0;  // disabled 64-key half
+      if (kMode == 2 && k != 0) {
+        if (a >= sink_lim && b <= wlo) k = 0;                      // between sinks and window, every lane
+        else if (!(b < sink_lim || a > whi)) k = 2;                // sink/window edge inside the chunk
+      }
+      cls[c] = k;
+    }
+  }
+  // Row max: per chunk two 3-input chains of 16 columns.
+  float mc[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    float m0 = -INFINITY, m1 = -INFINITY;
+    if (cls[c] == 1) {
+#pragma unroll
+      for (int e = 0; e < 16; e += 2) {
+        m0 = fmax3(m0, x[32 * c + e], x[32 * c + e + 1]);
+        m1 = fmax3(m1, x[32 * c + 16 + e], x[32 * c + 16 + e + 1]);
+      }
+    } else if (cls[c] == 2) {
+      auto xm = [&](int e) { return live(e) ? x[e] : -INFINITY; };
+#pragma unroll
+      for (int e = 0; e < 16; e += 2) {
+        m0 = fmax3(m0, xm(32 * c + e), xm(32 * c + e + 1));
+        m1 = fmax3(m1, xm(32 * c + 16 + e), xm(32 * c + 16 + e + 1));
+      }
+    }
+    mc[c] = fmaxf(m0, m1);
+  }
+  const float mt = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
+  const float mts = mt * scale_log2;
+  float f = 1.f;
+  if (mts > m_ref + kRescaleLog2) {
+    f = ex2(m_ref - mts);  // 0 while m_ref is still -inf
+    l *= f;
+    m_ref = mts;
+  }
+  // The exponentials start once this warp holds its sub-partition's MUFU turn; `sub` takes
+  // a zero that only exists after the wait, so no exponential is scheduled before it.
+  const float sub = ((m_ref == -INFINITY) ? 0.f : m_ref) + tok.acquire();
+  const uint64_t scale2 = f2_pack(scale_log2, scale_log2), nsub2 = f2_pack(-sub, -sub);
+  uint64_t l2 = f2_pack(0.f, 0.f);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    if (cls[c] == 0) {
+#pragma unroll
+      for (int e = 32 * c; e < 32 * c + 32; e += 2) pk[e / 2] = 0u;
+    } else if (cls[c] == 1) {
+#pragma unroll
+      for (int e = 32 * c; e < 32 * c + 32; e += 2) {
+        const uint64_t t2 = f2_fma(f2_pack(x[e], x[e + 1]), scale2, nsub2);
+        float p0, p1;
+        if (kPolyEvery > 0 && (e / 2) % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
+          ex2_pair_fma(t2, p0, p1);
+        } else {
+          float t0, t1;
+          f2_unpack(t2, t0, t1);
+          p0 = ex2(t0);
+          p1 = ex2(t1);
+        }
+        l2 = f2_add(l2, f2_pack(p0, p1));
+        pk[e / 2] = pack_bf16x2(p0, p1);
+      }
+    } else {
+#pragma unroll
+      for (int e = 32 * c; e < 32 * c + 32; e += 2) {
+        float t0, t1;
+        f2_unpack(f2_fma(f2_pack(x[e], x[e + 1]), scale2, nsub2), t0, t1);
+        const float e0 = ex2(t0), e1 = ex2(t1);
+        const float p0 = live(e) ? e0 : 0.f, p1 = live(e + 1) ? e1 : 0.f;
+        l2 = f2_add(l2, f2_pack(p0, p1));
+        pk[e / 2] = pack_bf16x2(p0, p1);
+      }
+    }
+  }
+  float la, lb;
+  f2_unpack(l2, la, lb);
+  l += la + lb;
+  tok.release(l);   // after the last exponential (the row sum depends on all of them)
+  return f;
+}
+
 // Row `row` of P into the K-major, 128-byte-swizzled tile at p_tile: keys 64b..64b+63
 // in box b, 16-byte chunk c of a row at chunk position c ^ (row % 8).
 __device__ __forceinline__ void store_p_row(uint32_t p_tile, int row, const uint32_t (&pk)[BN / 2]) {

@@ -283,7 +283,7 @@ hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           if (hb == 3 && ct < I.T)
             f = softmax_tile<0>(x, 0, 0, 0, p.scale_log2, m_ref, l, pk, turn);
           else
-            f = softmax_tile<3>(x, i - ct * BN, hb, 0, p.scale_log2, m_ref, l, pk, turn);
+            f = softmax_tile_chunked<3>(x, i - ct * BN, hb, 0, p.scale_log2, m_ref, l, pk, turn);
         } else if (tile_needs_mask(p, I.kind, I.T, ct)) {
           const int lim = i - ct * BN;
           if (kind_el == EA_STREAMING)
