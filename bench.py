@@ -35,13 +35,15 @@ DEFAULT_WORKLOAD = "llama3-8b-s32k-streaming"
 
 # DRAM bytes (read + write) of one attention launch from an ncu capture, keyed by the
 # hash of the kernel's sources: a changed kernel reports traffic null until re-measured.
-ATTN_SOURCES = ("sparse_gqa_attention_b200/csrc/ea_attn_tc.cu", "sparse_gqa_attention_b200/csrc/ea_common.cuh",
+ATTN_SOURCES = ("sparse_gqa_attention_b200/csrc/ea_attn_tc.cu", "sparse_gqa_attention_b200/csrc/ea_attn_tc.cuh",
+                "sparse_gqa_attention_b200/csrc/ea_common.cuh",
                 "sparse_gqa_attention_b200/csrc/ea_sm100.cuh")   # the block-128 kernel the default workload runs
 ATTN_TRAFFIC = {  # source hash -> {workload: bytes per launch}
     "0296169ffe64f919": {"llama3-8b-s32k-streaming": 588227584 + 242138624},
     "7f7dafa317af8ef7": {"llama3-8b-s32k-streaming": 592338944 + 243713536},
     "c9ec1a166bddf719": {"llama3-8b-s32k-streaming": 572987648 + 234234880},
     "d295b6f17472de2e": {"llama3-8b-s32k-streaming": 581203968 + 235314688},
+    "c69a5f23f33afc52": {"llama3-8b-s32k-streaming": 584922368 + 236055040},
 }
 
 def attn_source_hash():
