@@ -117,10 +117,11 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (!ok) break;
         int idx = (int)atomicAdd(hdr + kWsClaim / 4, 1u);
         if (idx >= n_items) idx = -1;
-        ring[e] = idx;
+        Item I{};
+        if (idx >= 0) I = load_item(items, idx, p, head_mode, H_kv, G);
+        put_item(ring + e * kItemWords, idx, I);
         mbar_arrive(c.bar(B_IFULL + e));
         if (idx < 0) break;
-        const Item I = load_item(items, idx, p, head_mode, H_kv, G);
         if (I.n == 0) continue;
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
@@ -173,9 +174,8 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       };
       ItemRing ir{reinterpret_cast<volatile int*>(gbase + OFF_IRING), 0};
       while (ok) {
-        const int idx = ir.next(c, true);
-        if (idx < 0) break;
-        const Item I = load_item(items, idx, p, head_mode, H_kv, G);
+        Item I;
+        if (ir.next(c, true, I) < 0) break;
         if (I.n == 0) continue;
         ok = wait(c, c.bar(B_QFULL + 0), q_use[0] & 1);
         ++q_use[0];
@@ -201,9 +201,8 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       bool ok = true;
       ItemRing ir{reinterpret_cast<volatile int*>(gbase + OFF_IRING), 0};
       while (ok) {
-        const int idx = ir.next(c, true);
-        if (idx < 0) break;
-        const Item I = load_item(items, idx, p, head_mode, H_kv, G);
+        Item I;
+        if (ir.next(c, true, I) < 0) break;
         if (I.n == 0) continue;
         ++kv;                                         // K(0)
         for (int jj = 0; jj < I.n && ok; ++jj) {
@@ -240,11 +239,11 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     turn.theirs = c.bar(B_TOK + 4 * (1 - s) + warp % 4);
     ItemRing ir{reinterpret_cast<volatile int*>(gbase + OFF_IRING), 0};
     while (ok) {
-      const int idx = ir.next(c, false);   // every lane reads the entry, then lane 0 releases it
+      Item I;
+      const int idx = ir.next(c, false, I);   // every lane reads the entry, then lane 0 releases it
       __syncwarp();
       if (lane == 0 && idx >= 0) mbar_arrive(c.bar(B_IEMPTY + ((ir.k - 1) & 1)));
       if (idx < 0) break;
-      const Item I = load_item(items, idx, p, head_mode, H_kv, G);
       if (I.n == 0 || (s == 1 && !I.two)) continue;
       turn.on = I.two;
       turn.ok = true;
@@ -324,20 +323,20 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const int h_q = I.h * G + 2 * I.pr + s;
       __nv_bfloat16* orow = o + (((size_t)I.b * S + i_out) * H_q + h_q) * HD;
+      {
+        uint32_t r[HD];   // the whole O row in one TMEM round trip
 #pragma unroll
-      for (int q4 = 0; q4 < HD / 32; ++q4) {
-        uint32_t r[32];
-        tmem_ld32(lane_addr + col_o(s) + 32 * q4, r);
+        for (int q4 = 0; q4 < HD / 32; ++q4) tmem_ld32(lane_addr + col_o(s) + 32 * q4, r + 32 * q4);
         tmem_ld_wait();
         if (i_out < S) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
+          for (int e = 0; e < HD; e += 8) {
             uint4 w;
             w.x = pack_bf16x2(__uint_as_float(r[e]) * inv, __uint_as_float(r[e + 1]) * inv);
             w.y = pack_bf16x2(__uint_as_float(r[e + 2]) * inv, __uint_as_float(r[e + 3]) * inv);
             w.z = pack_bf16x2(__uint_as_float(r[e + 4]) * inv, __uint_as_float(r[e + 5]) * inv);
             w.w = pack_bf16x2(__uint_as_float(r[e + 6]) * inv, __uint_as_float(r[e + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + 32 * q4 + e) = w;
+            *reinterpret_cast<uint4*>(orow + e) = w;
           }
         }
       }

@@ -38,8 +38,9 @@ enum : int {
 };
 constexpr uint32_t OFF_TMEM = OFF_BAR + N_BAR * 8;
 constexpr uint32_t OFF_ABORT = OFF_TMEM + 4;
-constexpr uint32_t OFF_IRING = OFF_ABORT + 4;          // 2 claimed item indices
-constexpr uint32_t kSmemBytes = OFF_IRING + 8 + 1024;  // + slack to align the base to 1024
+constexpr uint32_t OFF_IRING = OFF_ABORT + 4;          // 2 claimed items, kItemWords ints each
+constexpr int kItemWords = 12;
+constexpr uint32_t kSmemBytes = OFF_IRING + 2 * kItemWords * 4 + 1024;  // + slack to align the base to 1024
 // Roles that read every claimed item: Q K^T issuer, P V issuer and the 8 softmax warps.
 constexpr uint32_t kItemReaders = 10;
 static_assert(kSmemBytes <= 232448, "shared memory beyond the 227 KB a CTA may use");
@@ -98,17 +99,41 @@ struct Item {
 
 // Work items are claimed at run time: the producer takes the next index of the cost-sorted
 // list (longest first) from a counter in the workspace whenever its CTA can start another
-// item, and passes it to the other roles through a 2-entry ring in shared memory; -1 ends
-// the list.  Greedy longest-first claiming keeps the CTAs' finishing times close.
+// item, decodes it (load_item: the item word, the head's routed kind, its live-tile range)
+// and passes the decoded item to the other roles through a 2-entry ring in shared memory,
+// so that they start the item without global loads of their own; index -1 ends the list.
+// Greedy longest-first claiming keeps the CTAs' finishing times close.
+__device__ __forceinline__ void put_item(volatile int* e, int idx, const Item& I) {
+  e[0] = idx; e[1] = I.b; e[2] = I.h; e[3] = I.t; e[4] = I.T; e[5] = I.pr; e[6] = I.kind; e[7] = I.n;
+  e[8] = I.sink_end; e[9] = I.win_lo; e[10] = (int)I.csr_beg; e[11] = (int)(I.csr_beg >> 32) * 2 + (I.two ? 1 : 0);
+}
+__device__ __forceinline__ int get_item(const volatile int* e, Item& I) {
+  I.b = e[1]; I.h = e[2]; I.t = e[3]; I.T = e[4]; I.pr = e[5]; I.kind = e[6]; I.n = e[7];
+  I.sink_end = e[8]; I.win_lo = e[9];
+  const int hi = e[11];
+  I.two = (hi & 1) != 0;
+  I.csr_beg = (long long)(unsigned)e[10] | ((long long)(hi >> 1) << 32);
+  return e[0];
+}
 struct ItemRing {
-  volatile int* slot;   // 2 entries
+  volatile int* slot;   // 2 entries of kItemWords ints
   int k;                // items read so far
-  // Next item index for a reader role (-1: done or aborted).  `arrive` is true for the one
+  // Next item for a reader role (index -1: done or aborted).  `arrive` is true for the one
   // thread of the role that signals the entry as read.
-  __device__ int next(const Ctx& c, bool arrive) {
+  __device__ int next(const Ctx& c, bool arrive, Item& I) {
     const int e = k & 1;
     const bool ok = wait(c, c.bar(B_IFULL + e), (k >> 1) & 1);
-    const int idx = ok ? slot[e] : -1;
+    const int idx = ok ? get_item(slot + e * kItemWords, I) : -1;
+    if (ok && arrive) mbar_arrive(c.bar(B_IEMPTY + e));
+    ++k;
+    return idx;
+  }
+  // The index alone, for a ring whose producer publishes indices before decoding them (the
+  // block-64 kernel: there every role walks the item's layout rows itself, in parallel).
+  __device__ int next_idx(const Ctx& c, bool arrive) {
+    const int e = k & 1;
+    const bool ok = wait(c, c.bar(B_IFULL + e), (k >> 1) & 1);
+    const int idx = ok ? slot[e * kItemWords] : -1;
     if (ok && arrive) mbar_arrive(c.bar(B_IEMPTY + e));
     ++k;
     return idx;

@@ -114,7 +114,7 @@ hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         if (!ok) break;
         int idx = (int)atomicAdd(hdr + kWsClaim / 4, 1u);
         if (idx >= n_items) idx = -1;
-        ring[e] = idx;
+        ring[e * kItemWords] = idx;
         mbar_arrive(c.bar(B_IFULL + e));
         if (idx < 0) break;
         const Item I = load_item<true>(items, idx, p, head_mode, H_kv, G);
@@ -172,7 +172,7 @@ hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       };
       ItemRing ir{reinterpret_cast<volatile int*>(gbase + OFF_IRING), 0};
       while (ok) {
-        const int idx = ir.next(c, true);
+        const int idx = ir.next_idx(c, true);
         if (idx < 0) break;
         const Item I = load_item<true>(items, idx, p, head_mode, H_kv, G);
         if (I.n == 0) continue;
@@ -200,7 +200,7 @@ hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       bool ok = true;
       ItemRing ir{reinterpret_cast<volatile int*>(gbase + OFF_IRING), 0};
       while (ok) {
-        const int idx = ir.next(c, true);
+        const int idx = ir.next_idx(c, true);
         if (idx < 0) break;
         const Item I = load_item<true>(items, idx, p, head_mode, H_kv, G);
         if (I.n == 0) continue;
@@ -239,7 +239,7 @@ hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     turn.theirs = c.bar(B_TOK + 4 * (1 - s) + warp % 4);
     ItemRing ir{reinterpret_cast<volatile int*>(gbase + OFF_IRING), 0};
     while (ok) {
-      const int idx = ir.next(c, false);   // every lane reads the entry, then lane 0 releases it
+      const int idx = ir.next_idx(c, false);   // every lane reads the entry, then lane 0 releases it
       __syncwarp();
       if (lane == 0 && idx >= 0) mbar_arrive(c.bar(B_IEMPTY + ((ir.k - 1) & 1)));
       if (idx < 0) break;
