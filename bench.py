@@ -44,6 +44,7 @@ ATTN_TRAFFIC = {  # source hash -> {workload: bytes per launch}
     "c9ec1a166bddf719": {"llama3-8b-s32k-streaming": 572987648 + 234234880},
     "d295b6f17472de2e": {"llama3-8b-s32k-streaming": 581203968 + 235314688},
     "c69a5f23f33afc52": {"llama3-8b-s32k-streaming": 584922368 + 236055040},
+    "3d97ab8c0a397417": {"llama3-8b-s32k-streaming": 588211456 + 234348544},
 }
 
 def attn_source_hash():
