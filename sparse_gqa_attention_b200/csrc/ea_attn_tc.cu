@@ -32,7 +32,8 @@
 //               registers, then - once the previous P V product is done - rescales
 //               O in TMEM when the max was raised and writes P as bf16 into shared
 //               memory (the K-major swizzled layout the MMA reads); finally divides
-//               O by the row sum and stores bf16 rows.
+//               O by the row sum, stages the bf16 rows in its own rows of P_s and
+//               writes them out as whole 256-byte rows.
 // TMEM: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512) fp32 columns.  Shared
 // memory: Q0 Q1 | P0 P1 | K/V ring x3 (32 KB each) | barriers.
 #include <atomic>
@@ -248,7 +249,6 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       turn.on = I.two;
       turn.ok = true;
       const int i = I.T * BM + row;        // query position in the sequence
-      const int i_out = I.t * BM + row;    // row of q and o in this call
       const int kind_el = I.kind == EA_STREAMING ? EA_STREAMING : EA_FULL;
       float m_ref = -INFINITY, l = 0.f;
       for (int jj = 0; jj < I.n; ++jj) {
@@ -322,24 +322,34 @@ hybrid_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       fence_after_sync();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const int h_q = I.h * G + 2 * I.pr + s;
-      __nv_bfloat16* orow = o + (((size_t)I.b * S + i_out) * H_q + h_q) * HD;
       {
-        uint32_t r[HD];   // the whole O row in one TMEM round trip
+        // O rows scaled by 1/l, staged as bf16 in this warp's 32 rows of P_s (free: the item's
+        // last P V product is done), then written as whole 256-byte rows: lanes 0-15 one
+        // row's 16-byte chunks, lanes 16-31 the next row's.
+        uint32_t r[HD];
 #pragma unroll
         for (int q4 = 0; q4 < HD / 32; ++q4) tmem_ld32(lane_addr + col_o(s) + 32 * q4, r + 32 * q4);
         tmem_ld_wait();
-        if (i_out < S) {
+        uint32_t pk[BN / 2];
 #pragma unroll
-          for (int e = 0; e < HD; e += 8) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(r[e]) * inv, __uint_as_float(r[e + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(r[e + 2]) * inv, __uint_as_float(r[e + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(r[e + 4]) * inv, __uint_as_float(r[e + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(r[e + 6]) * inv, __uint_as_float(r[e + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + e) = w;
-          }
+        for (int e = 0; e < HD; e += 2) pk[e / 2] = pack_bf16x2(__uint_as_float(r[e]) * inv, __uint_as_float(r[e + 1]) * inv);
+        store_p_row(p_tile, row, pk);
+      }
+      __syncwarp();
+      {
+        const int cc = lane & 15;
+#pragma unroll 4
+        for (int j = 0; j < 16; ++j) {
+          const int rr = (warp % 4) * 32 + 2 * j + (lane >> 4);
+          const uint32_t a = p_tile + (uint32_t)(cc >> 3) * kBoxBytes + (uint32_t)rr * 128u +
+                             (uint32_t)(((cc & 7) ^ (rr & 7)) << 4);
+          uint4 v4;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v4.x), "=r"(v4.y), "=r"(v4.z), "=r"(v4.w) : "r"(a));
+          const int io = I.t * BM + rr;
+          if (io < S) *reinterpret_cast<uint4*>(o + (((size_t)I.b * S + io) * H_q + h_q) * HD + cc * 8) = v4;
         }
       }
+      __syncwarp();
       fence_before_sync();
     }
   }
