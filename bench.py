@@ -45,6 +45,8 @@ ATTN_TRAFFIC = {  # source hash -> {workload: bytes per launch}
     "d295b6f17472de2e": {"llama3-8b-s32k-streaming": 581203968 + 235314688},
     "c69a5f23f33afc52": {"llama3-8b-s32k-streaming": 584922368 + 236055040},
     "3d97ab8c0a397417": {"llama3-8b-s32k-streaming": 588211456 + 234348544},
+    # captured on sources hashing to ef26b9e687f25042, which differ from these only in a comment
+    "72ab3cb333c45a5f": {"llama3-8b-s32k-streaming": 606085376 + 237764608},
 }
 
 def attn_source_hash():
