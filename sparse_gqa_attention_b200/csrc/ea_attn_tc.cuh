@@ -140,10 +140,13 @@ struct ItemRing {
   }
 };
 
-// kBlock64: the block-64 kernel's items (block-sparse heads walk the union of two CSR rows).
+// kBlock64: the block-64 kernel's items (block-sparse heads walk the union of two CSR rows;
+// their live-tile count is read from the schedule's cost pass, `cost`, instead of walking
+// the rows once more).
 template <bool kBlock64 = false>
 __device__ __forceinline__ Item load_item(const int4* items, int idx, const PatternDev& p,
-                                          const int32_t* head_mode, int H_kv, int G) {
+                                          const int32_t* head_mode, int H_kv, int G,
+                                          const int* cost = nullptr) {
   const int4 w = items[idx];
   Item I;
   I.b = w.x; I.h = w.y; I.t = w.z; I.pr = w.w;
@@ -156,7 +159,7 @@ __device__ __forceinline__ Item load_item(const int4* items, int idx, const Patt
     stream_ranges(p, I.kind, I.T, I.sink_end, I.win_lo);
     I.n = I.sink_end + max(0, I.T - I.win_lo + 1);
   } else if (kBlock64 && bs64_kind(p, I.kind)) {
-    I.n = n_live_tiles(p, I.kind, H_kv, I.b, I.h, I.T);
+    I.n = cost[((size_t)I.b * H_kv + I.h) * p.n_qt + I.t];
   } else if (I.kind == EA_BLOCK_SPARSE) {
     long long a, e;
     csr_row(p, H_kv, I.b, I.h, I.T, a, e);

@@ -54,7 +54,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o,
                       const int32_t* __restrict__ head_mode, const PatternDev p, int S, int H_q, int H_kv,
-                      const int4* __restrict__ items, uint32_t* __restrict__ hdr, int inject_stall) {
+                      const int4* __restrict__ items, uint32_t* __restrict__ hdr, int inject_stall,
+                      const int* __restrict__ cost) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -117,7 +118,7 @@ hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         ring[e * kItemWords] = idx;
         mbar_arrive(c.bar(B_IFULL + e));
         if (idx < 0) break;
-        const Item I = load_item<true>(items, idx, p, head_mode, H_kv, G);
+        const Item I = load_item<true>(items, idx, p, head_mode, H_kv, G, cost);
         if (I.n == 0) continue;
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
@@ -174,7 +175,7 @@ hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       while (ok) {
         const int idx = ir.next_idx(c, true);
         if (idx < 0) break;
-        const Item I = load_item<true>(items, idx, p, head_mode, H_kv, G);
+        const Item I = load_item<true>(items, idx, p, head_mode, H_kv, G, cost);
         if (I.n == 0) continue;
         ok = wait(c, c.bar(B_QFULL + 0), q_use[0] & 1);
         ++q_use[0];
@@ -202,7 +203,7 @@ hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       while (ok) {
         const int idx = ir.next_idx(c, true);
         if (idx < 0) break;
-        const Item I = load_item<true>(items, idx, p, head_mode, H_kv, G);
+        const Item I = load_item<true>(items, idx, p, head_mode, H_kv, G, cost);
         if (I.n == 0) continue;
         ++kv;                                         // K(0)
         for (int jj = 0; jj < I.n && ok; ++jj) {
@@ -243,7 +244,7 @@ hybrid_attn_tc64_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       __syncwarp();
       if (lane == 0 && idx >= 0) mbar_arrive(c.bar(B_IEMPTY + ((ir.k - 1) & 1)));
       if (idx < 0) break;
-      const Item I = load_item<true>(items, idx, p, head_mode, H_kv, G);
+      const Item I = load_item<true>(items, idx, p, head_mode, H_kv, G, cost);
       if (I.n == 0 || (s == 1 && !I.two)) continue;
       turn.on = I.two;
       turn.ok = true;
@@ -387,7 +388,8 @@ ea_status launch_attn_tc64(const void* q, const void* k, const void* v, void* o,
   const int inject = take_inject_stall() ? 1 : 0;
   kern<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), head_mode, pat, S, H_q,
                                            H_kv, reinterpret_cast<const int4*>(ws + items_off),
-                                           reinterpret_cast<uint32_t*>(ws), inject);
+                                           reinterpret_cast<uint32_t*>(ws), inject,
+                                           reinterpret_cast<const int*>(ws + attn_costs_offset(B, S, H_q, H_kv)));
   return cudaGetLastError() == cudaSuccess ? EA_OK : EA_ERR_CUDA;
 }
 

@@ -17,6 +17,9 @@ ea_status launch_router_pool(const void* hidden, ea_dtype dtype, int B, int S, i
                              void* workspace, cudaStream_t st);
 
 size_t attn_workspace_bytes(int B, int S, int H_q, int H_kv);
+// Offset in the attention workspace of the schedule's live-tile counts: int32 per
+// (b, h_kv, query tile of the call), index (b * H_kv + h) * n_qt + t.
+size_t attn_costs_offset(int B, int S, int H_q, int H_kv);
 int n_pairs(int H_q, int H_kv);
 ea_status launch_schedule(const int32_t* head_mode, const PatternDev& pat, int B, int S, int H_q, int H_kv,
                           void* workspace, cudaStream_t st);

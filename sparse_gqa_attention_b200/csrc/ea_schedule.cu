@@ -181,6 +181,8 @@ static size_t costs_offset(int B, int S, int H_q, int H_kv) {
   return items_offset(B) + n_items * sizeof(int4);
 }
 
+size_t attn_costs_offset(int B, int S, int H_q, int H_kv) { return costs_offset(B, S, H_q, H_kv); }
+
 size_t attn_workspace_bytes(int B, int S, int H_q, int H_kv) {
   return costs_offset(B, S, H_q, H_kv) + ((size_t)B * H_kv * cdiv(S, kTile) * 4 + 255) / 256 * 256;
 }
