@@ -125,19 +125,17 @@ EA_API ea_status ea_router_pool(const void* hidden, ea_dtype dtype, int B, int S
                                 float* hbar, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Router with library-owned scratch.  The paper has no counterpart: this is an
- * interface for callers that cannot allocate device memory — a runtime or plugin
- * host that owns every device allocation, or code running while a stream is
- * captured (cudaMalloc is rejected during a global-mode capture and may
- * synchronise the device).  Same arguments and outputs as ea_router, without
- * the workspace: the scratch is a fixed EA_ROUTER_STATIC_SCRATCH_BYTES array
+ * interface for callers that cannot allocate device memory, such as a runtime or
+ * plugin host that owns every device allocation.  Same arguments and outputs as
+ * ea_router, without the workspace: the scratch is a fixed EA_ROUTER_STATIC_SCRATCH_BYTES array
  * inside the library, held on every GPU that loads it until the process exits.
  * It allocates nothing (no cudaMalloc, cudaFree or allocating library call).
  * Problems whose scratch (ea_router_workspace_size) exceeds the array return
  * EA_ERR_INVALID_ARG before any launch.  The first call in each context (per
  * device; again after a device reset or in a caller's own context) looks up
- * the array's device address; make that first call before any stream
- * capture.  All calls share the array: calls that overlap on the GPU race, so
- * order them on one stream.  Nothing in the array needs to start at zero. */
+ * the array's device address with a host-side runtime query.  All calls share
+ * the array: calls that overlap on the GPU race, so order them on one stream.
+ * Nothing in the array needs to start at zero. */
 #define EA_ROUTER_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
 EA_API ea_status ea_router_static_scratch(const void* hidden, ea_dtype dtype, int B, int S, int D, int H_kv,
                                           int d, const ea_router_weights* weights,

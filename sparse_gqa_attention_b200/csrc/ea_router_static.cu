@@ -1,20 +1,18 @@
 // ea_router_static.cu — ea_router_static_scratch: the router with scratch memory that
 // the library owns, for callers that cannot allocate device memory.
 //
-// Some callers of this router cannot call cudaMalloc: an inference runtime or plugin
-// host that hands out all device memory through its own allocator, or code that runs
-// while a stream is being captured (a global-mode capture rejects cudaMalloc, and
-// cudaMalloc/cudaFree can synchronise the device).  This entry point takes the same
-// inputs and outputs as ea_router but keeps its pooling partial sums and pooled
-// hidden states in a fixed array compiled into the library, so it allocates nothing.
+// Some callers of this router cannot call cudaMalloc, for instance an inference runtime
+// or plugin host that hands out all device memory through its own allocator.  This
+// entry point takes the same inputs and outputs as ea_router but keeps its pooling
+// partial sums and pooled hidden states in a fixed array compiled into the library, so
+// it allocates nothing.
 //
 // The array is a file-scope __device__ variable: every GPU that loads the library holds
 // kStaticScratchBytes of it until the process exits.  Host code cannot use the array's
 // name as a device address, so the first call on each device looks the address up with
 // cudaGetSymbolAddress (that device current) and caches it together with the context it
 // was found in; a later call in another context (after a device reset, or from a caller's
-// own context) looks it up again.  That first call in a context should come before any
-// stream capture.  All calls share the one array, so calls whose kernels
+// own context) looks it up again.  All calls share the one array, so calls whose kernels
 // overlap on the GPU (different streams, or different host threads) race on it; order
 // them on one stream.  Nothing in it needs to start at zero: every byte a call reads was
 // written earlier in the same call.

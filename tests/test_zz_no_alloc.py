@@ -1,7 +1,7 @@
 """The router entry point that allocates nothing (GPU).
 
-ea_router_static_scratch serves callers that cannot call cudaMalloc (a runtime
-that owns every device allocation, or code running under stream capture): it
+ea_router_static_scratch serves callers that cannot call cudaMalloc (such as a
+runtime that owns every device allocation): it
 keeps its scratch in a fixed array inside the library instead of a caller
 workspace.  Its decisions and logits must match ea_router's on the same inputs,
 on two calls in a row (the second call reuses the array the first one left
