@@ -76,3 +76,16 @@ def test_reference_arm_under_torchrun_prints_once():
     assert len(lines) == 1
     _check(lines[0], "small-mixed-g4-s1000")
     assert lines[0]["n_gpus"] == 2
+
+
+def test_config_states_how_l2_reuse_is_avoided():
+    """Timed steps need inputs larger than L2 (126 MB) or a flush: every bench workload's inputs
+    exceed L2, and a parity-size case says that it fits instead of claiming otherwise."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as wl
+    for name in ("llama3-8b-s32k-streaming", "qwen-g7-s64k-blocksparse", "llama3-8b-b4-s16k-mixed",
+                 "llama3-8b-s128k-sweep", "llama3-8b-s32k-xassa"):
+        assert bench.l2_note(wl.WORKLOADS[name]).startswith("inputs larger than L2"), name
+    small = bench.l2_note(wl.WORKLOADS["small-mixed-g4-s1000"])
+    assert small.startswith("inputs fit in L2") and "not a bench line" in small
