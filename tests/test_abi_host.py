@@ -83,6 +83,37 @@ def test_router_argument_checks(lib):
                          None, ws, 8, None) == abi.EA_ERR_INVALID_ARG            # workspace too small
 
 
+def test_router_weight_alignment_is_checked(lib):
+    """The router stages W_k and the MLP weights with 16-byte asynchronous copies, so each
+    weight matrix must start on a 16-byte boundary; a misaligned one is refused on the host."""
+    ws = ctypes.c_void_p(0x100000)
+    prm = abi.RouterParams(100)
+    for i in (0, 1, 3, 5, 7):   # w_k, w_t1, w_t2, w_r1, w_o
+        ptrs = [FAKE] * 9
+        ptrs[i] = ctypes.c_void_p(0x10004)
+        w = abi.RouterWeights(*ptrs)
+        assert lib.ea_router(FAKE, abi.EA_DT_F32, 1, 300, 256, 2, 128, ctypes.byref(w), ctypes.byref(prm), FAKE,
+                             None, ws, 1 << 30, None) == abi.EA_ERR_INVALID_ARG, i
+
+
+@pytest.mark.parametrize("case", [
+    dict(hidden=None),                       # no input
+    dict(hbar=None),                         # no output
+    dict(B=0), dict(S=0), dict(D=0),
+    dict(D=100),                             # D % 8 != 0 for bf16
+    dict(hidden=ctypes.c_void_p(0x10008)),   # not 16-byte aligned
+    dict(dtype=7),                           # unknown dtype
+    dict(ws_bytes=8),                        # workspace too small
+    dict(ws=ctypes.c_void_p(0x100010)),      # workspace not 256-byte aligned
+])
+def test_router_pool_argument_checks(lib, case):
+    c = dict(hidden=FAKE, dtype=abi.EA_DT_BF16, B=1, S=300, D=256, n=100, hbar=FAKE, ws=ctypes.c_void_p(0x100000),
+             ws_bytes=1 << 30)
+    c.update(case)
+    assert lib.ea_router_pool(c["hidden"], c["dtype"], c["B"], c["S"], c["D"], c["n"], c["hbar"], c["ws"],
+                              c["ws_bytes"], None) == abi.EA_ERR_INVALID_ARG
+
+
 @pytest.mark.parametrize("q_offset,S_q,S_k,expect", [
     (64, 100, 1000, abi.EA_ERR_INVALID_ARG),     # chunks start on a multiple of 128
     (896, 200, 1000, abi.EA_ERR_INVALID_ARG),    # rows past the keys
